@@ -1,0 +1,312 @@
+/*
+ * CPU oracle for 8-bit quantized softmax attention (SageAttention).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only the test-suite, the smoke check and the
+ * benchmark's CPU-baseline leg may load this library.  The product path
+ * (the CUDA library and its Python binding) never calls into it, and the two
+ * share no code, headers, tables or constants.
+ *
+ * It follows the SageAttention article ("又快又准，即插即用！清华8比特量化
+ * Attention"), method section:
+ *   - "对 K 进行平滑处理": K <- K - mean(K), which leaves softmax(QK^T) unchanged;
+ *   - "对 Q, K 进行分块 INT8 量化": INT8 quantization of Q and K per
+ *     FlashAttention-sized block, INT8 matmul with an INT32 accumulator;
+ *   - "对 P, V 采用 FP16 数据类型的矩阵乘法累加器": P and V kept in FP16.
+ *
+ * Readings where the article is silent (each is a plain choice, listed with
+ * its reason in the design notes of the repository):
+ *   mean axis   the mean runs over the token axis, one value per channel and
+ *               per (batch, kv head), over all Lk tokens.  Only a vector that
+ *               is constant across tokens leaves each softmax row unchanged.
+ *   mean value  sum = sum_t int64(K[t,c] * 2^24) (exact, fp16 values are
+ *               multiples of 2^-24), m = float(double(sum) * 2^-24 / double(Lk)).
+ *   quantizer   symmetric, range +-127, per block a = max|x|,
+ *               r = fl32(127 / a), q = clamp(rne(fl32(x * r)), -127, 127),
+ *               scale = fl32(a / 127).  An all-zero block gives q = 0 and
+ *               scale = 0.  For K, x = fl32(float(K) - m).
+ *   blocks      Q blocks are 128 rows, K blocks 64 rows, each spanning all d
+ *               channels of one (batch, head); the last block holds the
+ *               remaining rows only.
+ *   sm_scale    folded into Q's scale together with log2(e):
+ *               c = fl32(double(sm_scale) * log2(e)), q_scale = fl32(scale * c),
+ *               so the softmax runs in base 2.
+ *   P rounding  the quantized-path simulation rounds every
+ *               p = exp2(s - rowmax) to fp16 and accumulates in fp64.
+ *   causal      bottom-right aligned: key j is visible to query i iff
+ *               j <= i + Lk - Lq; a row with no visible key outputs 0.
+ *
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -fno-fast-math -shared -fPIC.
+ * All float arithmetic below is IEEE binary32/binary64 with round-to-nearest.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------ fp16 */
+
+/* fp16 bit pattern -> exact double. */
+double oracle_half_to_double(uint16_t h)
+{
+    int sign = h >> 15;
+    int e = (h >> 10) & 0x1f;
+    int m = h & 0x3ff;
+    double v;
+    if (e == 0)
+        v = ldexp((double)m, -24);               /* subnormal or zero */
+    else if (e == 31)
+        v = m ? NAN : INFINITY;
+    else
+        v = ldexp((double)(m | 0x400), e - 25);  /* (1.m) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* double -> fp16 bit pattern, round to nearest, ties to even. */
+uint16_t oracle_double_to_half(double x)
+{
+    uint16_t sign = signbit(x) ? 0x8000 : 0;
+    if (isnan(x))
+        return 0x7e00;
+    double a = fabs(x);
+    if (a < ldexp(1.0, -14)) {
+        /* subnormal range: value = n * 2^-24, n in [0, 1024]; n = 1024 is
+           the smallest normal, whose encoding is exactly 0x0400 */
+        double n = nearbyint(ldexp(a, 24));
+        return sign | (uint16_t)n;
+    }
+    int e2;
+    frexp(a, &e2);              /* a in [2^(e2-1), 2^e2) */
+    int E = e2 - 1;             /* unbiased exponent */
+    double n = nearbyint(ldexp(a, 10 - E));   /* significand in [1024, 2048] */
+    if (n == 2048.0) {
+        n = 1024.0;
+        E += 1;
+    }
+    if (E > 15)
+        return sign | 0x7c00;   /* overflow to infinity */
+    return sign | (uint16_t)(((E + 15) << 10) | ((int)n - 1024));
+}
+
+/* --------------------------------------------------------------- K mean */
+
+/* Per-(batch, kv head, channel) mean of K over all Lk tokens (smoothing
+ * step).  k: fp16 bits [B, Hkv, Lk, d]; k_mean: float [B, Hkv, d]. */
+void oracle_k_mean(const uint16_t *k, int B, int Hkv, int Lk, int d, float *k_mean)
+{
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        for (int c = 0; c < d; ++c) {
+            int64_t sum = 0;
+            for (int t = 0; t < Lk; ++t) {
+                double v = oracle_half_to_double(k[((int64_t)bh * Lk + t) * d + c]);
+                sum += (int64_t)(v * 16777216.0);     /* exact integer */
+            }
+            double mean = ((double)sum * ldexp(1.0, -24)) / (double)Lk;
+            k_mean[(int64_t)bh * d + c] = (float)mean;
+        }
+    }
+}
+
+/* ------------------------------------------------------- block quantizer */
+
+/* Quantize one block of `rows` x `d` fp32 values to int8 with one scale.
+ * Returns fl32(a / 127) (0 for an all-zero block). */
+static float quant_block(const float *x, int rows, int d, int8_t *q)
+{
+    float a = 0.0f;
+    for (int i = 0; i < rows * d; ++i) {
+        float m = fabsf(x[i]);
+        if (m > a)
+            a = m;
+    }
+    if (a == 0.0f) {
+        memset(q, 0, (size_t)rows * d);
+        return 0.0f;
+    }
+    float r = 127.0f / a;
+    for (int i = 0; i < rows * d; ++i) {
+        float y = x[i] * r;
+        float t = nearbyintf(y);               /* ties to even */
+        if (t > 127.0f) t = 127.0f;
+        if (t < -127.0f) t = -127.0f;
+        q[i] = (int8_t)t;
+    }
+    return a / 127.0f;
+}
+
+/* Block quantization of Q and smoothed K.
+ *   q  fp16 [B, H, Lq, d]     -> q_i8 [B, H, Lq, d],  q_scale [B, H, ceil(Lq/128)]
+ *   k  fp16 [B, Hkv, Lk, d]   -> k_i8 [B, Hkv, Lk, d], k_scale [B, Hkv, ceil(Lk/64)]
+ *   k_mean [B, Hkv, d]        (written)
+ * smooth = 0 skips the mean subtraction (ablation only; k_mean is then 0). */
+void oracle_quant_qk(const uint16_t *q, const uint16_t *k, int B, int H, int Hkv,
+                     int Lq, int Lk, int d, double sm_scale, int smooth,
+                     int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale,
+                     float *k_mean)
+{
+    const int BQ = 128, BK = 64;
+    const int nqb = (Lq + BQ - 1) / BQ, nkb = (Lk + BK - 1) / BK;
+    const float c = (float)(sm_scale * 1.4426950408889634074);   /* log2(e) */
+
+    if (smooth)
+        oracle_k_mean(k, B, Hkv, Lk, d, k_mean);
+    else
+        for (int i = 0; i < B * Hkv * d; ++i) k_mean[i] = 0.0f;
+
+    float *buf = (float *)malloc(sizeof(float) * (size_t)BQ * d);
+    for (int bh = 0; bh < B * H; ++bh) {
+        for (int blk = 0; blk < nqb; ++blk) {
+            int r0 = blk * BQ, rows = Lq - r0 < BQ ? Lq - r0 : BQ;
+            const uint16_t *src = q + ((int64_t)bh * Lq + r0) * d;
+            for (int i = 0; i < rows * d; ++i)
+                buf[i] = (float)oracle_half_to_double(src[i]);
+            float s = quant_block(buf, rows, d, q_i8 + ((int64_t)bh * Lq + r0) * d);
+            q_scale[(int64_t)bh * nqb + blk] = s * c;
+        }
+    }
+    for (int bh = 0; bh < B * Hkv; ++bh) {
+        const float *m = k_mean + (int64_t)bh * d;
+        for (int blk = 0; blk < nkb; ++blk) {
+            int r0 = blk * BK, rows = Lk - r0 < BK ? Lk - r0 : BK;
+            const uint16_t *src = k + ((int64_t)bh * Lk + r0) * d;
+            for (int i = 0; i < rows; ++i)
+                for (int ch = 0; ch < d; ++ch)
+                    buf[i * d + ch] = (float)oracle_half_to_double(src[i * d + ch]) - m[ch];
+            k_scale[(int64_t)bh * nkb + blk] =
+                quant_block(buf, rows, d, k_i8 + ((int64_t)bh * Lk + r0) * d);
+        }
+    }
+    free(buf);
+}
+
+/* ------------------------------------------------------------ attention */
+
+static int64_t visible_keys(int i, int Lq, int Lk, int causal)
+{
+    if (!causal)
+        return Lk;
+    int64_t n = (int64_t)i + (Lk - Lq) + 1;
+    if (n < 0) n = 0;
+    if (n > Lk) n = Lk;
+    return n;
+}
+
+/* Simulation of the quantized forward pass, in the article's order:
+ * S = int32 sum of int8 products (exact), s = S * q_scale * k_scale (already
+ * in base-2 units), p = fp16(exp2(s - max s)), O = sum p v / sum p in fp64.
+ * rows: flat indices (b*H + h)*Lq + i to compute, or NULL for all rows.
+ * out: [n_rows, d] doubles (unrounded output). */
+void oracle_attn_quant_sim(const int8_t *q_i8, const int8_t *k_i8,
+                           const float *q_scale, const float *k_scale,
+                           const uint16_t *v, int B, int H, int Hkv, int Lq, int Lk,
+                           int d, int causal, const int64_t *rows, int64_t n_rows,
+                           double *out)
+{
+    const int nqb = (Lq + 127) / 128, nkb = (Lk + 63) / 64;
+    const int group = H / Hkv;
+    if (!rows)
+        n_rows = (int64_t)B * H * Lq;
+
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t flat = rows ? rows[r] : r;
+            int i = (int)(flat % Lq);
+            int64_t bh = flat / Lq;
+            int b = (int)(bh / H), h = (int)(bh % H);
+            int64_t bhk = (int64_t)b * Hkv + h / group;
+            double *o = out + r * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            int64_t nvis = visible_keys(i, Lq, Lk, causal);
+            if (nvis == 0)
+                continue;
+            const int8_t *qi = q_i8 + (bh * Lq + i) * d;
+            double sq = (double)q_scale[bh * nqb + i / 128];
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nvis; ++j) {
+                const int8_t *kj = k_i8 + (bhk * Lk + j) * d;
+                int32_t acc = 0;
+                for (int c = 0; c < d; ++c)
+                    acc += (int32_t)qi[c] * (int32_t)kj[c];
+                s[j] = (double)acc * sq * (double)k_scale[bhk * nkb + j / 64];
+                if (s[j] > mx) mx = s[j];
+            }
+            double l = 0.0;
+            for (int64_t j = 0; j < nvis; ++j) {
+                double p = oracle_half_to_double(oracle_double_to_half(exp2(s[j] - mx)));
+                l += p;
+                const uint16_t *vj = v + (bhk * Lk + j) * d;
+                for (int c = 0; c < d; ++c)
+                    o[c] += p * oracle_half_to_double(vj[c]);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= l;
+        }
+        free(s);
+    }
+}
+
+/* Full-precision attention straight from the fp16 inputs, no smoothing and no
+ * quantization: O = softmax(sm_scale * Q K^T + mask) V in fp64. */
+void oracle_attn_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                      int B, int H, int Hkv, int Lq, int Lk, int d, int causal,
+                      double sm_scale, const int64_t *rows, int64_t n_rows, double *out)
+{
+    const int group = H / Hkv;
+    if (!rows)
+        n_rows = (int64_t)B * H * Lq;
+
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double *qi = (double *)malloc(sizeof(double) * (size_t)d);
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t flat = rows ? rows[r] : r;
+            int i = (int)(flat % Lq);
+            int64_t bh = flat / Lq;
+            int b = (int)(bh / H), h = (int)(bh % H);
+            int64_t bhk = (int64_t)b * Hkv + h / group;
+            double *o = out + r * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            int64_t nvis = visible_keys(i, Lq, Lk, causal);
+            if (nvis == 0)
+                continue;
+            for (int c = 0; c < d; ++c)
+                qi[c] = oracle_half_to_double(q[(bh * Lq + i) * d + c]);
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nvis; ++j) {
+                const uint16_t *kj = k + (bhk * Lk + j) * d;
+                double acc = 0.0;
+                for (int c = 0; c < d; ++c)
+                    acc += qi[c] * oracle_half_to_double(kj[c]);
+                s[j] = acc * sm_scale;
+                if (s[j] > mx) mx = s[j];
+            }
+            double l = 0.0;
+            for (int64_t j = 0; j < nvis; ++j) {
+                double p = exp(s[j] - mx);
+                l += p;
+                const uint16_t *vj = v + (bhk * Lk + j) * d;
+                for (int c = 0; c < d; ++c)
+                    o[c] += p * oracle_half_to_double(vj[c]);
+            }
+            for (int c = 0; c < d; ++c) o[c] /= l;
+        }
+        free(s);
+        free(qi);
+    }
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
