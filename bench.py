@@ -1,0 +1,390 @@
+"""Benchmark of the 8-bit quantized attention forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload 1..5]
+
+A step is one pass of the whole hot path over the workload: K mean + Q/K
+quantization (sage_quant_qk) and the fused attention kernel
+(sage_attn_fwd_prequant) -- exactly what sage_attn_fwd runs, with the scratch
+preallocated so the timed region holds only kernels.  Inputs are seeded
+synthetic fp16 tensors resident in HBM before timing; L2 is flushed (256 MiB
+write) before every timed step, outside the step's CUDA events.
+
+Metric: TOPS = 4 * d * (unmasked query/key pairs) / step time, the QK^T and
+PV work counted at 2*d each.  ``e2e`` is the same metric through the public
+host-buffer call (sage_attn_fwd_host: H2D of q/k/v, forward pass, D2H of the
+output, all inside the timed region).  ``roofline`` reports the attention
+kernel against the combined tensor roofline: QK at the INT8 peak and PV at the
+FP16 peak, t_roof = 2*d*pairs/P_int8 + 2*d*pairs/P_fp16, with P_fp16 the
+measured bf16 peak and P_int8 = 2 x P_fp16 (nominal dense ratio).
+
+Multi-GPU (torchrun, one process per GPU): every rank runs the same workload
+on its own GPU (the path shards by batch and head with no exchange, so this
+is weak scaling); value = all ranks' ops / the slowest rank's time.
+``--impl reference`` times the CPU oracle (the only reference this path has)
+on a bounded row sample per step, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_quantized_attention_mean_b200 import inputs  # noqa: E402
+
+METRIC = "quantized attention fwd TOPS at 1 B200 and % of INT8/FP16 tensor roofline"
+DEFAULT_WORKLOAD = 2
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+
+# DRAM traffic of one attention launch from an ncu capture, valid only for the
+# kernel source it was taken on (sha256 of attn.cu); otherwise reported null.
+NCU_TRAFFIC = {}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def attn_source_hash():
+    p = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc", "attn.cu")
+    with open(p, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+# ------------------------------------------------------------ clock sampler
+
+class ClockSampler:
+    """Samples SM clock, power and throttle reasons via NVML while running."""
+
+    REASONS = {
+        0x0000000000000001: "gpu_idle",
+        0x0000000000000002: "applications_clocks_setting",
+        0x0000000000000004: "sw_power_cap",
+        0x0000000000000008: "hw_slowdown",
+        0x0000000000000020: "sw_thermal_slowdown",
+        0x0000000000000040: "hw_thermal_slowdown",
+        0x0000000000000080: "hw_power_brake_slowdown",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples = []
+        self.max_mhz = None
+        self.period = period_s
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            try:  # NVML indices ignore CUDA_VISIBLE_DEVICES; match by UUID
+                uuid = "GPU-" + str(torch.cuda.get_device_properties(device_index).uuid)
+                self._h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - depends on the box
+            self._nvml = None
+            self.error = str(e)
+
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                reasons = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                util = nv.nvmlDeviceGetUtilizationRates(self._h).gpu
+                self.samples.append((mhz, reasons, util))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._nvml is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+
+    def summary(self):
+        if self._nvml is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": getattr(self, "error", "nvml unavailable")}
+        busy = [s for s in self.samples if s[2] > 0] or self.samples
+        mask = 0
+        for s in busy:
+            mask |= s[1]
+        reasons = [n for bit, n in self.REASONS.items() if mask & bit and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(busy)}
+
+
+# ---------------------------------------------------------- distributed
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def time_oracle_sample(w, q, k, v, n_rows, seed):
+    """Oracle on a bounded sample: full Q/K quantization + n_rows query rows
+    of the quantized-path simulation.  Returns (est_full_seconds, info)."""
+    import oracle
+    sm = float(np.float32(w.sm_scale))
+    t0 = time.perf_counter()
+    qk = oracle.quant_qk(q, k, sm)
+    t_quant = time.perf_counter() - t0
+    rng = np.random.default_rng(seed)
+    rows = np.sort(rng.choice(w.B * w.H * w.Lq, size=n_rows, replace=False)).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.attn_quant_sim(*qk[:4], v, w.causal, rows=rows)
+    t_attn = time.perf_counter() - t0
+    i = rows % w.Lq
+    vis = np.minimum(w.Lk, np.maximum(0, i + (w.Lk - w.Lq) + 1)) if w.causal else np.full(n_rows, w.Lk)
+    sample_pairs = float(vis.sum())
+    est = t_quant + t_attn * (w.pairs() / sample_pairs)
+    return est, {"t_quant_s": t_quant, "t_attn_sample_s": t_attn, "rows": n_rows,
+                 "sample_pairs": sample_pairs, "cores": oracle.num_threads()}
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return 0
+    q, k, v = inputs.make_inputs(w)
+    ops = 4.0 * w.d * w.pairs()
+    rows = args.ref_rows
+    times = []
+    info = None
+    for step in range(args.warmup + args.steps):
+        est, info = time_oracle_sample(w, q, k, v, rows, seed=step)
+        if step >= args.warmup:
+            times.append(est)
+    t = float(np.mean(times))
+    value = ops / t / 1e12
+    sample = (f"per step: oracle Q/K quantization of the full workload + quantized-path "
+              f"simulation of {rows} random query rows, time extrapolated to all "
+              f"{w.pairs()} query/key pairs")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64 (int8 codes, int32 dot products)",
+        "data": "synthetic (seeded numpy, fp16)",
+        "config": dict(w.describe(), l2="n/a (CPU)"),
+        "cpu_baseline": {"value": value, "unit": "TOPS", "cores": info["cores"],
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- ours
+
+def run_ours(args, w):
+    import torch
+    import bit_quantized_attention_mean_b200 as sage
+
+    world, rank, local = dist_setup()
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+
+    qn, kn, vn = inputs.make_inputs(w)
+    sm = float(np.float32(w.sm_scale))
+    q = torch.from_numpy(qn).to(dev)
+    k = torch.from_numpy(kn).to(dev)
+    v = torch.from_numpy(vn).to(dev)
+    out = torch.empty_like(q)
+    B, H, Hkv, Lq, Lk, d = w.B, w.H, w.Hkv, w.Lq, w.Lk, w.d
+    q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
+    k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
+    q_scale = torch.empty((B, H, -(-Lq // 128)), dtype=torch.float32, device=dev)
+    k_scale = torch.empty((B, Hkv, -(-Lk // 64)), dtype=torch.float32, device=dev)
+    k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, sage.sage_quant_workspace_size(B, Hkv, Lk, d)), dtype=torch.uint8,
+                     device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    launches = 0
+
+    def step():
+        nonlocal launches
+        sage.sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, workspace=ws,
+                           stream=stream)
+        launches += sage.sage_last_launch_count()
+        ev_mid = torch.cuda.Event(enable_timing=True)
+        ev_mid.record(stream)
+        sage.sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, w.causal,
+                                    stream=stream)
+        launches += sage.sage_last_launch_count()
+        return ev_mid
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    sage.sage_check_device_status(stream)
+
+    n = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    mids = []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    launches = 0
+    with ClockSampler(local) as clocks:
+        for i in range(n):
+            flush.zero_()
+            evs[i][0].record(stream)
+            mids.append(step())
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    sage.sage_check_device_status(stream)
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    attn_ms = [m.elapsed_time(b) for m, (a, b) in zip(mids, evs)]
+    total_ms = float(sum(step_ms))
+    attn_avg_ms = float(sum(attn_ms) / n)
+    quant_avg_ms = float(sum(m0.elapsed_time(m) for (m0, _), m in zip(evs, mids)) / n)
+
+    # e2e through the host-buffer entry point (pinned memory)
+    hq = torch.from_numpy(qn).pin_memory()
+    hk = torch.from_numpy(kn).pin_memory()
+    hv = torch.from_numpy(vn).pin_memory()
+    hout = torch.empty(qn.shape, dtype=torch.float16).pin_memory()
+    e2e_steps = max(1, min(n, args.e2e_steps))
+    for _ in range(2):
+        sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+    torch.cuda.synchronize(dev)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(e2e_steps)]
+    for a, b in e2e_ev:
+        a.record(stream)
+        sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    sage.sage_check_device_status(stream)
+    e2e_ms = float(sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps)
+
+    stats = torch.tensor([total_ms, attn_avg_ms, e2e_ms, quant_avg_ms], dtype=torch.float64,
+                         device=dev)
+    nl = torch.tensor([launches], dtype=torch.int64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
+        torch.distributed.all_reduce(nl, op=torch.distributed.ReduceOp.SUM)
+    total_ms, attn_avg_ms, e2e_ms, quant_avg_ms = stats.tolist()
+
+    result = None
+    if rank == 0:
+        ops = 4.0 * d * w.pairs()
+        ms_per_step = total_ms / n
+        value = world * ops / (ms_per_step * 1e-3) / 1e12
+        peaks = load_peaks()
+        p16 = float(peaks["bf16_tflops"])
+        p8 = INT8_OVER_FP16 * p16
+        t_roof_ms = (2.0 * d * w.pairs() / (p8 * 1e12) + 2.0 * d * w.pairs() / (p16 * 1e12)) * 1e3
+        peak_eff = ops / (t_roof_ms * 1e-3) / 1e12
+        achieved = ops / (attn_avg_ms * 1e-3) / 1e12
+        traffic = None
+        if NCU_TRAFFIC.get("attn_sha") == attn_source_hash() and \
+                NCU_TRAFFIC.get("workload") == w.name:
+            traffic = NCU_TRAFFIC.get("bytes_per_launch")
+        quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d
+        result = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": n, "warmup": args.warmup, "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "int8 QK^T (int32 acc) + fp16 PV (fp32 acc)",
+            "data": "synthetic (seeded numpy N(0,1)/t4 fp16, per-channel K offsets)",
+            "config": dict(w.describe(), l2="flushed before every timed step (256 MiB write)",
+                           parallelism=f"replicas x{world} (shard by batch/head)"),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
+                         "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
+                         "kernel": "sage_attn_fwd_kernel",
+                         "peak_note": (f"combined INT8/FP16 roofline: P_fp16 = {p16} TFLOP/s "
+                                       f"({peaks.get('source')} bf16 burst), P_int8 = "
+                                       f"{INT8_OVER_FP16} x P_fp16 (nominal ratio)")},
+            "kernel_ms": {"attention": attn_avg_ms, "quant": quant_avg_ms},
+            "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
+            "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                    "h2d_bytes_per_step": int(qn.nbytes + kn.nbytes + vn.nbytes),
+                    "d2h_bytes_per_step": int(qn.nbytes)},
+            "gpu_launches": int(nl.item()),
+            "clocks": clocks.summary(),
+        }
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        est, info = time_oracle_sample(w, qn, kn, vn, args.cpu_rows, seed=0)
+        result["cpu_baseline"] = {
+            "value": 4.0 * d * w.pairs() / est / 1e12, "unit": "TOPS",
+            "cores": info["cores"], "kind": "oracle",
+            "sample": (f"oracle Q/K quantization of the full workload "
+                       f"({info['t_quant_s']:.2f} s) + quantized-path simulation of "
+                       f"{info['rows']} random query rows ({info['t_attn_sample_s']:.2f} s), "
+                       f"extrapolated to all query/key pairs")}
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    w = inputs.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

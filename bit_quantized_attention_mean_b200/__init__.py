@@ -1,0 +1,33 @@
+"""B200-native 8-bit quantized attention (SageAttention forward pass).
+
+A thin Python binding over the C ABI of ``libsage_b200.so`` (declared in
+``include/sage.h``).  Every function here only checks and marshals arguments
+(torch CUDA tensors -> device pointers, torch's current stream) and calls the
+library; all arithmetic runs in the library's sm_100a kernels.  There is no
+CPU or PyTorch fallback: if the library is missing, every call raises.
+
+Exported names mirror the C ABI:
+    sage_quant_qk, sage_attn_fwd, sage_attn_fwd_prequant,
+    sage_quant_workspace_size, sage_attn_workspace_size,
+    sage_check_device_status, sage_status_string, sage_last_launch_count
+plus two conveniences that allocate outputs: ``quant_qk`` and ``attention``.
+"""
+from __future__ import annotations
+
+from ._lib import (  # noqa: F401
+    SageError,
+    SYMBOLS,
+    library_path,
+    load_library,
+    sage_attn_fwd,
+    sage_attn_fwd_host,
+    sage_attn_fwd_prequant,
+    sage_attn_workspace_size,
+    sage_check_device_status,
+    sage_last_launch_count,
+    sage_quant_qk,
+    sage_quant_workspace_size,
+    sage_status_string,
+    quant_qk,
+    attention,
+)

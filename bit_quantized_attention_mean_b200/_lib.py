@@ -1,0 +1,228 @@
+"""ctypes marshalling for libsage_b200.so (C ABI in include/sage.h).
+
+Argument marshalling only: shape/dtype/device checks, torch tensor -> device
+pointer, torch's current CUDA stream -> cudaStream_t.  No arithmetic happens
+here and there is no fallback path: a missing library raises on first use.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libsage_b200.so")
+_lock = threading.Lock()
+_lib = None
+
+# Every symbol include/sage.h declares.
+SYMBOLS = (
+    "sage_quant_qk",
+    "sage_quant_workspace_size",
+    "sage_attn_fwd_prequant",
+    "sage_attn_fwd",
+    "sage_attn_fwd_host",
+    "sage_attn_workspace_size",
+    "sage_check_device_status",
+    "sage_status_string",
+    "sage_last_launch_count",
+)
+
+STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
+          3: "SAGE_ERR_CUDA", 4: "SAGE_ERR_TIMEOUT"}
+
+
+class SageError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where} failed: {STATUS.get(status, status)}")
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libsage_b200.so (raises if it was not built)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(
+                f"{_LIB_PATH} is missing: build it with "
+                "`python -m bit_quantized_attention_mean_b200.build` (no fallback exists)")
+        lib = ctypes.CDLL(_LIB_PATH)
+        P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        lib.sage_quant_qk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, Z, P]
+        lib.sage_quant_qk.restype = I
+        lib.sage_quant_workspace_size.argtypes = [I, I, I, I]
+        lib.sage_quant_workspace_size.restype = Z
+        lib.sage_attn_fwd_prequant.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
+        lib.sage_attn_fwd_prequant.restype = I
+        lib.sage_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
+        lib.sage_attn_fwd.restype = I
+        lib.sage_attn_fwd_host.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
+        lib.sage_attn_fwd_host.restype = I
+        lib.sage_attn_workspace_size.argtypes = [I, I, I, I, I, I]
+        lib.sage_attn_workspace_size.restype = Z
+        lib.sage_check_device_status.argtypes = [P]
+        lib.sage_check_device_status.restype = I
+        lib.sage_status_string.argtypes = [I]
+        lib.sage_status_string.restype = ctypes.c_char_p
+        lib.sage_last_launch_count.argtypes = []
+        lib.sage_last_launch_count.restype = I
+        _lib = lib
+        return lib
+
+
+def _stream(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _dev(t, dtype, name, shape=None):
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(t.shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise SageError(status, where)
+
+
+def _dims(q, k):
+    B, H, Lq, d = q.shape
+    Bk, Hkv, Lk, dk = k.shape
+    if Bk != B or dk != d:
+        raise ValueError("q and k disagree on batch or head dim")
+    return B, H, Hkv, Lq, Lk, d
+
+
+# --------------------------------------------------------------- C ABI names
+
+def sage_status_string(status: int) -> str:
+    return load_library().sage_status_string(int(status)).decode()
+
+
+def sage_last_launch_count() -> int:
+    return load_library().sage_last_launch_count()
+
+
+def sage_quant_workspace_size(B, Hkv, Lk, d) -> int:
+    return load_library().sage_quant_workspace_size(B, Hkv, Lk, d)
+
+
+def sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
+    return load_library().sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d)
+
+
+def sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
+                  workspace=None, stream=None):
+    """Smooth K and quantize Q/K per block into the given output tensors."""
+    import torch
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    nqb, nkb = -(-Lq // 128), -(-Lk // 64)
+    args = [
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(q_i8, torch.int8, "q_i8", q.shape), _dev(k_i8, torch.int8, "k_i8", k.shape),
+        _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
+        _dev(k_scale, torch.float32, "k_scale", (B, Hkv, nkb)),
+        _dev(k_mean, torch.float32, "k_mean", (B, Hkv, d)),
+    ]
+    if workspace is None:
+        ws, wsb = ctypes.c_void_p(0), 0
+    else:
+        ws, wsb = _dev(workspace, torch.uint8, "workspace"), workspace.numel()
+    _check(lib.sage_quant_qk(*args, B, H, Hkv, Lq, Lk, d, float(sm_scale), ws, wsb,
+                             _stream(stream)), "sage_quant_qk")
+
+
+def sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, causal, stream=None):
+    """Attention kernel on pre-quantized Q/K (fp16 V, fp16 out)."""
+    import torch
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q_i8, k_i8)
+    nqb, nkb = -(-Lq // 128), -(-Lk // 64)
+    _check(lib.sage_attn_fwd_prequant(
+        _dev(q_i8, torch.int8, "q_i8"), _dev(k_i8, torch.int8, "k_i8"),
+        _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
+        _dev(k_scale, torch.float32, "k_scale", (B, Hkv, nkb)),
+        _dev(v, torch.float16, "v", k_i8.shape), _dev(out, torch.float16, "out", q_i8.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, _stream(stream)), "sage_attn_fwd_prequant")
+
+
+def sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=None):
+    """Whole forward pass on fp16 device tensors, output written into `out`."""
+    import torch
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    _check(lib.sage_attn_fwd(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
+        "sage_attn_fwd")
+
+
+def sage_attn_fwd_host(q, k, v, out, causal, sm_scale, stream=None):
+    """Whole forward pass on HOST fp16 tensors (pinned for async copies)."""
+    import torch
+    lib = load_library()
+    for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.float16 \
+                or not t.is_contiguous():
+            raise ValueError(f"{name}: expected a contiguous fp16 host tensor")
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    if tuple(v.shape) != tuple(k.shape) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("v must match k and out must match q")
+    _check(lib.sage_attn_fwd_host(
+        ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
+        ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
+        "sage_attn_fwd_host")
+
+
+def sage_check_device_status(stream=None):
+    """Synchronize the stream and raise if a kernel's bounded wait gave up."""
+    _check(load_library().sage_check_device_status(_stream(stream)),
+           "sage_check_device_status")
+
+
+# --------------------------------------------------------- conveniences
+
+def quant_qk(q, k, sm_scale, stream=None):
+    """Allocate outputs and run sage_quant_qk.
+    Returns (q_i8, k_i8, q_scale, k_scale, k_mean) as CUDA tensors."""
+    import torch
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    dev = q.device
+    q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
+    k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
+    q_scale = torch.empty((B, H, -(-Lq // 128)), dtype=torch.float32, device=dev)
+    k_scale = torch.empty((B, Hkv, -(-Lk // 64)), dtype=torch.float32, device=dev)
+    k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+    sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, stream=stream)
+    return q_i8, k_i8, q_scale, k_scale, k_mean
+
+
+def attention(q, k, v, causal=False, sm_scale=None, stream=None):
+    """Allocate the output and run sage_attn_fwd; returns the fp16 output."""
+    import torch
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    out = torch.empty_like(q)
+    sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=stream)
+    return out

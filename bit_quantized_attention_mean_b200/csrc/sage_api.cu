@@ -1,0 +1,220 @@
+// sage_api.cu -- the C ABI declared in include/sage.h: host-side argument
+// validation, scratch management and dispatch to the sm_100a kernels.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+
+#include "../../include/sage.h"
+#include "sage_internal.h"
+
+namespace {
+
+thread_local int g_last_launches = 0;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+sage_status check_shape(int B, int H, int Hkv, int Lq, int Lk, int d) {
+  if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1) return SAGE_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return SAGE_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+  // every element offset and grid size must fit the kernels' index types
+  const long long qn = (long long)B * H * Lq, kn = (long long)B * Hkv * Lk;
+  if (qn * d > (1LL << 40) || kn * d > (1LL << 40)) return SAGE_ERR_INVALID_ARG;
+  if (qn / 128 + 1 > 0x7fffffffLL || kn / 64 + 1 > 0x7fffffffLL) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+sage_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  if (major != 10 || minor != 0) return SAGE_ERR_UNSUPPORTED;  // built for sm_100a only
+  return SAGE_OK;
+}
+
+float fold_constant(float sm_scale) {
+  // c = fl32(double(sm_scale) * log2(e)); folded into the Q scales
+  return (float)((double)sm_scale * 1.4426950408889634074);
+}
+
+size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
+
+struct AttnWorkspace {
+  size_t q_i8, k_i8, q_scale, k_scale, k_mean, part, total;
+};
+
+AttnWorkspace attn_workspace_layout(int B, int H, int Hkv, int Lq, int Lk, int d) {
+  AttnWorkspace w;
+  const size_t nqb = (size_t)(Lq + 127) / 128, nkb = (size_t)(Lk + 63) / 64;
+  size_t off = 0;
+  w.q_i8 = off;    off += round_up((size_t)B * H * Lq * d);
+  w.k_i8 = off;    off += round_up((size_t)B * Hkv * Lk * d);
+  w.q_scale = off; off += round_up((size_t)B * H * nqb * 4);
+  w.k_scale = off; off += round_up((size_t)B * Hkv * nkb * 4);
+  w.k_mean = off;  off += round_up((size_t)B * Hkv * d * 4);
+  w.part = off;    off += round_up(sage::quant_workspace_bytes(B, Hkv, Lk, d));
+  w.total = off;
+  return w;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* sage_status_string(sage_status s) {
+  switch (s) {
+    case SAGE_OK: return "SAGE_OK";
+    case SAGE_ERR_INVALID_ARG: return "SAGE_ERR_INVALID_ARG";
+    case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
+    case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
+    case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+  }
+  return "SAGE_ERR_UNKNOWN";
+}
+
+int sage_last_launch_count(void) { return g_last_launches; }
+
+size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d) {
+  if (B < 1 || Hkv < 1 || Lk < 1 || (d != 64 && d != 128)) return 0;
+  return sage::quant_workspace_bytes(B, Hkv, Lk, d);
+}
+
+size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
+  if (check_shape(B, H, Hkv, Lq, Lk, d) != SAGE_OK) return 0;
+  return attn_workspace_layout(B, H, Hkv, Lq, Lk, d).total;
+}
+
+sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale,
+                          float* k_scale, float* k_mean, int B, int H, int Hkv, int Lq, int Lk,
+                          int d, float sm_scale, void* workspace, size_t workspace_bytes,
+                          void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!q || !k || !q_i8 || !k_i8 || !q_scale || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8) ||
+      !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(k_mean))
+    return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  const size_t need = sage::quant_workspace_bytes(B, Hkv, Lk, d);
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  sage::QuantArgs a{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
+                    q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale)};
+  int launches = 0;
+  cudaError_t e = sage::launch_quant(a, s, &launches);
+  if (!workspace && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_attn_fwd_prequant(const int8_t* q_i8, const int8_t* k_i8, const float* q_scale,
+                                   const float* k_scale, const void* v, void* out, int B, int H,
+                                   int Hkv, int Lq, int Lk, int d, int causal, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v || !out) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(q_scale) || !aligned16(k_scale))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  sage::AttnArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
+                   static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1};
+  int launches = 0;
+  cudaError_t e = sage::launch_attn(a, static_cast<cudaStream_t>(stream), &launches);
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
+                          int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
+                          void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const AttnWorkspace w = attn_workspace_layout(B, H, Hkv, Lq, Lk, d);
+  char* ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  int8_t* q_i8 = reinterpret_cast<int8_t*>(ws + w.q_i8);
+  int8_t* k_i8 = reinterpret_cast<int8_t*>(ws + w.k_i8);
+  float* q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+  float* k_scale = reinterpret_cast<float*>(ws + w.k_scale);
+  float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
+  sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
+                     q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
+                     fold_constant(sm_scale)};
+  int launches = 0;
+  cudaError_t e = sage::launch_quant(qa, s, &launches);
+  if (e == cudaSuccess) {
+    sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
+                      static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1};
+    e = sage::launch_attn(aa, s, &launches);
+  }
+  if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
+                               void* out_host, int B, int H, int Hkv, int Lq, int Lk, int d,
+                               int causal, float sm_scale, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_host) return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t qb = (size_t)B * H * Lq * d * 2, kb = (size_t)B * Hkv * Lk * d * 2;
+  char* buf = nullptr;
+  const size_t total = round_up(qb) * 2 + round_up(kb) * 2;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&buf), total, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  char* dq = buf;
+  char* dout = dq + round_up(qb);
+  char* dk = dout + round_up(qb);
+  char* dv = dk + round_up(kb);
+  cudaError_t e = cudaMemcpyAsync(dq, q_host, qb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, kb, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, kb, cudaMemcpyHostToDevice, s);
+  int launches = 0;
+  if (e == cudaSuccess) {
+    st = sage_attn_fwd(dq, dk, dv, dout, B, H, Hkv, Lq, Lk, d, causal, sm_scale, stream);
+    launches = g_last_launches;
+    if (st != SAGE_OK) e = cudaErrorUnknown;
+  }
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, dout, qb, cudaMemcpyDeviceToHost, s);
+  if (cudaFreeAsync(buf, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  if (st != SAGE_OK) return st;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_check_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGE_ERR_CUDA;
+  int v = 0;
+  if (sage::read_and_clear_device_status(&v) != cudaSuccess) return SAGE_ERR_CUDA;
+  return v != 0 ? SAGE_ERR_TIMEOUT : SAGE_OK;
+}
+
+}  // extern "C"

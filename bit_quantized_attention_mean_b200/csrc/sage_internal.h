@@ -1,0 +1,50 @@
+// sage_internal.h -- launcher interfaces shared by the library's translation
+// units (not part of the public ABI; see include/sage.h for that).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#define SAGE_Q_BLOCK_ROWS 128
+#define SAGE_K_BLOCK_ROWS 64
+
+namespace sage {
+
+struct QuantArgs {
+  const __half* q;
+  const __half* k;
+  int8_t* q_i8;
+  int8_t* k_i8;
+  float* q_scale;
+  float* k_scale;
+  float* k_mean;
+  void* workspace;  // quant_workspace_bytes() of scratch (int64 partial sums)
+  int B, H, Hkv, Lq, Lk, d;
+  float c;          // fl32(double(sm_scale) * log2(e)), folded into q_scale
+};
+
+struct AttnArgs {
+  const int8_t* q_i8;
+  const int8_t* k_i8;
+  const float* q_scale;
+  const float* k_scale;
+  const __half* v;
+  __half* out;
+  int B, H, Hkv, Lq, Lk, d;
+  bool causal;
+};
+
+size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d);
+
+// Each launcher adds the number of kernels it launched to *launches and
+// returns the first CUDA error (cudaSuccess when every launch was accepted).
+cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st, int* launches);
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches);
+
+// Device status word written by kernels whose bounded waits gave up.
+cudaError_t read_and_clear_device_status(int* value);
+
+}  // namespace sage

@@ -1,0 +1,157 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) 8-bit quantized attention library
+ * (libsage_b200.so).
+ *
+ * The operation is the forward pass of SageAttention as its article states it
+ * ("SageAttention: Accurate 8-Bit Attention for Plug-and-play Inference
+ * Acceleration", method section):
+ *   1. K smoothing: K <- K - mean(K), the mean taken over the token axis, one
+ *      value per channel (softmax(QK^T) = softmax(Q(K - mean K)^T));
+ *   2. per-block INT8 quantization of Q and K at FlashAttention tile size
+ *      (Q blocks of 128 rows, K blocks of 64 rows, one fp32 scale each);
+ *   3. S = Q_i8 K_i8^T with INT32 accumulation, dequantized by q_scale*k_scale;
+ *   4. online (tiled) softmax in base 2 (sm_scale*log2(e) is folded into
+ *      q_scale);
+ *   5. O = P V with P and V kept in FP16 (FP32 accumulation on this GPU).
+ *
+ * Conventions for every call:
+ *   - Tensors are CUDA device pointers to contiguous row-major arrays,
+ *     [B, heads, L, d] ("HND"), owned by the caller.  The library never frees
+ *     or retains them.  fp16 arguments are IEEE binary16 (`__half`), passed as
+ *     `void*`.
+ *   - Every pointer must be 16-byte aligned.  Q/K/V/out must not overlap.
+ *   - d must be 64 or 128; H % Hkv == 0 (query head h reads kv head
+ *     h / (H / Hkv)); Lq, Lk >= 1; B, H, Hkv >= 1; sm_scale > 0 and finite.
+ *   - Causal masking is bottom-right aligned: key j is visible to query i iff
+ *     j <= i + Lk - Lq.  A query row with no visible key produces zeros.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Calls are asynchronous on that stream.
+ *   - Argument errors are detected on the host before anything is launched
+ *     and return SAGE_ERR_INVALID_ARG / SAGE_ERR_UNSUPPORTED.  A failed launch
+ *     or allocation returns SAGE_ERR_CUDA.  Errors inside a kernel (a bounded
+ *     wait that gave up) are recorded in a device status word, read by
+ *     sage_check_device_status().
+ *   - Inputs must be finite; NaN/Inf inputs give unspecified outputs.
+ */
+#ifndef SAGE_B200_H
+#define SAGE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size */
+    SAGE_ERR_UNSUPPORTED = 2,   /* d not in {64,128}, or no sm_100 device */
+    SAGE_ERR_CUDA = 3,          /* a CUDA launch, allocation or copy failed */
+    SAGE_ERR_TIMEOUT = 4        /* a kernel's bounded wait gave up */
+} sage_status;
+
+/* Quantization block sizes (rows per block along the token axis). */
+#define SAGE_Q_BLOCK 128
+#define SAGE_K_BLOCK 64
+
+/*
+ * sage_quant_qk -- steps 1-2: smoothing of K and per-block INT8 quantization.
+ *
+ *   q        fp16 [B, H, Lq, d]            (in)
+ *   k        fp16 [B, Hkv, Lk, d]          (in)
+ *   q_i8     int8 [B, H, Lq, d]            (out)
+ *   k_i8     int8 [B, Hkv, Lk, d]          (out) quantized K - mean(K)
+ *   q_scale  fp32 [B, H, ceil(Lq/128)]     (out) fl32(fl32(amax/127) * c),
+ *                                          c = fl32(double(sm_scale)*log2(e))
+ *   k_scale  fp32 [B, Hkv, ceil(Lk/64)]    (out) fl32(amax/127)
+ *   k_mean   fp32 [B, Hkv, d]              (out) mean of K over all Lk tokens
+ *   workspace, workspace_bytes: device scratch of at least
+ *            sage_quant_workspace_size(B, Hkv, Lk, d) bytes, or NULL/0 to let
+ *            the call allocate it with cudaMallocAsync on `stream`.
+ *
+ * Per block: a = max|x|, r = fl32(127/a), q = clamp(rne(fl32(x*r)), -127, 127);
+ * an all-zero block gives q = 0 and scale 0.  For K, x = fl32(float(K) - m),
+ * m = fl32(double(sum_t int64(K*2^24)) * 2^-24 / Lk), exact and
+ * order-independent, so results are bit-reproducible.
+ */
+SAGE_API sage_status sage_quant_qk(const void *q, const void *k,
+                          int8_t *q_i8, int8_t *k_i8,
+                          float *q_scale, float *k_scale, float *k_mean,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          float sm_scale, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/* Bytes of scratch sage_quant_qk needs (exact int64 partial sums of K). */
+SAGE_API size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d);
+
+/*
+ * sage_attn_fwd_prequant -- steps 3-5 on already-quantized Q/K: one fused
+ * kernel (TMA -> tcgen05 INT8 QK^T into tensor memory -> dequant + exp2
+ * online softmax -> FP16 P into tensor memory -> tcgen05 FP16 P.V).
+ *
+ *   q_i8, k_i8, q_scale, k_scale   as produced by sage_quant_qk
+ *   v     fp16 [B, Hkv, Lk, d]     (in)
+ *   out   fp16 [B, H, Lq, d]       (out) O = softmax(S) V, rounded to fp16
+ *   causal  0 or 1
+ * Needs no scratch memory.
+ */
+SAGE_API sage_status sage_attn_fwd_prequant(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, void *stream);
+
+/*
+ * sage_attn_fwd -- the whole forward pass (steps 1-5) on fp16 Q, K, V.
+ *   q fp16 [B, H, Lq, d], k/v fp16 [B, Hkv, Lk, d], out fp16 [B, H, Lq, d].
+ * Scratch (int8 Q/K, scales, mean, partial sums;
+ * sage_attn_workspace_size() bytes) is allocated with cudaMallocAsync on
+ * `stream` and released with cudaFreeAsync on the same stream.
+ */
+SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *out,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          int causal, float sm_scale, void *stream);
+
+/*
+ * sage_attn_fwd_host -- sage_attn_fwd on HOST buffers, for callers whose data
+ * lives in host memory.  q/k/v/out are host pointers with the layouts of
+ * sage_attn_fwd (pinned memory gives asynchronous copies; pageable memory
+ * works but the copies then block the calling thread).  On `stream` the call
+ * allocates device buffers (cudaMallocAsync), copies q, k, v to the device
+ * (one cudaMemcpyAsync each), runs the forward pass, copies the output back
+ * and frees the device buffers.  The host output is valid once `stream` has
+ * been synchronized; the host buffers must stay alive until then.
+ */
+SAGE_API sage_status sage_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
+                               void *out_host, int B, int H, int Hkv, int Lq, int Lk, int d,
+                               int causal, float sm_scale, void *stream);
+
+/* Bytes of scratch sage_attn_fwd allocates for one call. */
+SAGE_API size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
+
+/*
+ * sage_check_device_status -- synchronizes `stream`, then reports and clears
+ * the device status word: SAGE_ERR_TIMEOUT if any kernel launched since the
+ * last check gave up on a bounded wait (its outputs are then invalid),
+ * SAGE_ERR_CUDA if the synchronization itself failed, else SAGE_OK.
+ */
+SAGE_API sage_status sage_check_device_status(void *stream);
+
+/* Static, human-readable name of a status code. */
+SAGE_API const char *sage_status_string(sage_status s);
+
+/* Number of kernels the last successful call on this thread launched. */
+SAGE_API int sage_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H */
