@@ -69,7 +69,8 @@ struct AttnCfg {
   static constexpr int B_S_FULL = B_KV_EMPTY + STAGES;
   static constexpr int B_P_FULL = B_S_FULL + 2;
   static constexpr int B_O_DONE = B_P_FULL + 2;
-  static constexpr int B_TEARDOWN = B_O_DONE + 1;
+  static constexpr int B_O_FINAL = B_O_DONE + 1;
+  static constexpr int B_TEARDOWN = B_O_FINAL + 1;
   static constexpr int NUM_BARS = B_TEARDOWN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int USED = OFF_MISC + 16;
@@ -228,7 +229,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
             break;
           }
         }
-        if (ok) issue_pv(nkt - 1);
+        if (ok && issue_pv(nkt - 1)) umma_commit(&bars[C::B_O_FINAL]);
       }
       // every issued MMA must be complete before the tensor memory is freed
       umma_commit(&bars[C::B_TEARDOWN]);
@@ -280,6 +281,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         m_run = mt;
       }
       if (j > 0 && __any_sync(0xffffffffu, need)) {
+        // S_j's commit came after P V_{j-2} was issued, so O_DONE is at most
+        // one phase behind P V_{j-1}: the parity wait is unambiguous
         if (!warp_wait(&bars[C::B_O_DONE], (j - 1) & 1, abort_flag, 7)) {
           ok = false;
           break;
@@ -318,7 +321,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_arrive(&bars[C::B_P_FULL + bb]);
     }
     if (ok && nkt > 0) {
-      ok = warp_wait(&bars[C::B_O_DONE], (nkt - 1) & 1, abort_flag, 8);
+      // O_DONE may still be two phases behind here (only P V_{nkt-3} is known
+      // to be complete), so the final accumulator has its own one-shot barrier
+      ok = warp_wait(&bars[C::B_O_FINAL], 0, abort_flag, 8);
       tc_fence_after_sync();
     }
     if (ok) {

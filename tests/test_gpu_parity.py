@@ -56,7 +56,13 @@ def assert_close(gpu_f16, sim, fp64=None, what=""):
     assert c >= COS_SIM, f"{what}: cos vs simulation {c}"
     if fp64 is not None:
         c64 = cos(g, fp64)
-        assert c64 >= COS_FP64, f"{what}: cos vs fp64 {c64}"
+        # The fp64 gate measures the method, not the kernel.  Where the
+        # method's own simulation falls short of it (heavy-tailed inputs), the
+        # kernel must lose nothing relative to that simulation.
+        method = cos(sim, fp64)
+        floor = COS_FP64 if method >= COS_FP64 else method - 1e-4
+        print(f"{what}: cos vs sim {c:.6f}, vs fp64 {c64:.6f} (method {method:.6f})")
+        assert c64 >= floor, f"{what}: cos vs fp64 {c64} (method's own {method})"
 
 
 def gpu_quant(q, k, sm):
@@ -114,6 +120,31 @@ def test_attention_small_full_compare(shape):
     sim, _ = oracle.attention(q, k, v, causal, sm)
     ref = oracle.attn_fp64(q, k, v, causal, sm)
     assert_close(out, sim, ref, str(shape))
+
+
+MEDIUM = [
+    # every row compared; enough CTAs that two share each SM and the tensor
+    # core queue is long (short causal tiles finish while their last P V
+    # products are still in flight)
+    (1, 32, 32, 1024, 1024, 128, True),
+    (2, 16, 4, 768, 768, 128, True),
+    (1, 24, 24, 1024, 1024, 64, False),
+    (1, 32, 32, 640, 640, 64, True),
+]
+
+
+@pytest.mark.parametrize("shape", MEDIUM)
+def test_attention_medium_all_rows(shape):
+    B, H, Hkv, Lq, Lk, d, causal = shape
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=Lq + H, k_offset_sigma=2.0)
+    sm = float(np.float32(1 / math.sqrt(d)))
+    for _ in range(2):   # twice: also checks run-to-run identity under load
+        out = gpu_attention(q, k, v, causal, sm)
+        if _ == 0:
+            first = out
+    assert np.array_equal(first, out)
+    sim, _ = oracle.attention(q, k, v, causal, sm)
+    assert_close(out, sim, None, str(shape))
 
 
 def test_prequant_matches_whole_path():
