@@ -21,6 +21,8 @@ from ._lib import (  # noqa: F401
     load_library,
     sage_attn_fwd,
     sage_attn_fwd_host,
+    sage_attn_fwd_noalloc,
+    NOALLOC_SCRATCH_BYTES,
     sage_attn_fwd_prequant,
     sage_attn_workspace_size,
     sage_check_device_status,

@@ -26,6 +26,7 @@ SYMBOLS = (
     "sage_check_device_status",
     "sage_status_string",
     "sage_last_launch_count",
+    "sage_attn_fwd_noalloc",
 )
 
 STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
@@ -70,6 +71,8 @@ def load_library():
         lib.sage_check_device_status.restype = I
         lib.sage_status_string.argtypes = [I]
         lib.sage_status_string.restype = ctypes.c_char_p
+        lib.sage_attn_fwd_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
+        lib.sage_attn_fwd_noalloc.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -175,6 +178,33 @@ def sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=None):
         _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
         B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
         "sage_attn_fwd")
+
+
+NOALLOC_SCRATCH_BYTES = 64 << 20
+
+
+def sage_attn_fwd_noalloc(q, k, v, out, causal, sm_scale, stream=None):
+    """Whole forward pass without allocating device memory during the call.
+
+    For callers that cannot allocate at call time (a server that reserved its
+    memory budget up front, a plugin host without an allocator for the
+    library).  The library's scratch is one fixed 64 MiB device array shared by
+    all calls: order the calls on one stream, make the first call on a device
+    before any stream capture, and keep problems within the array
+    (sage_attn_workspace_size(...) <= 64 MiB), else SageError is raised."""
+    import torch
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    status = lib.sage_attn_fwd_noalloc(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream))
+    if status != 0:
+        need = lib.sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d)
+        if status == 1 and need > NOALLOC_SCRATCH_BYTES:
+            raise SageError(status, f"sage_attn_fwd_noalloc (needs {need} bytes of scratch, "
+                                    f"the fixed array holds {NOALLOC_SCRATCH_BYTES})")
+        raise SageError(status, "sage_attn_fwd_noalloc")
 
 
 def sage_attn_fwd_host(q, k, v, out, causal, sm_scale, stream=None):

@@ -133,6 +133,26 @@ SAGE_API sage_status sage_attn_fwd_host(const void *q_host, const void *k_host, 
                                void *out_host, int B, int H, int Hkv, int Lq, int Lk, int d,
                                int causal, float sm_scale, void *stream);
 
+/*
+ * sage_attn_fwd_noalloc -- sage_attn_fwd for callers that must not allocate
+ * device memory at call time (a serving process that reserved its whole
+ * memory budget at start-up and treats any later allocation as an error, or a
+ * plugin host that gives the library no allocator).  The article has no
+ * counterpart; this is a packaging variant of the same forward pass.
+ *   Arguments, layouts and results are those of sage_attn_fwd.  The scratch
+ *   lives in one fixed 64 MiB device array inside the library, reserved on
+ *   every GPU that loads that part of the library and held until exit.
+ *   Problems needing more scratch than that (sage_attn_workspace_size() >
+ *   64 MiB) return SAGE_ERR_INVALID_ARG without launching anything.
+ *   All calls share the array: calls whose kernels overlap on the GPU race
+ *   and give wrong results, so order them on one stream.  The first call on
+ *   each device looks the array up; make it before any stream capture begins.
+ *   Nothing in the array needs clearing between calls.
+ */
+SAGE_API sage_status sage_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                           void *out, int B, int H, int Hkv, int Lq, int Lk,
+                                           int d, int causal, float sm_scale, void *stream);
+
 /* Bytes of scratch sage_attn_fwd allocates for one call. */
 SAGE_API size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
 
