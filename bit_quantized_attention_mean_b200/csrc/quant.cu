@@ -2,20 +2,26 @@
 // sm_100a (SageAttention article, method section: "对 K 进行平滑处理" and
 // "对 Q, K 进行分块 INT8 量化").
 //
-// Three launches on the caller's stream, all HBM-bound streaming kernels:
-//   1. kmean_and_quant_q: CTAs [0, n_chunk_ctas) reduce 256-token chunks of K
-//      to exact int64 fixed-point column sums (units of 2^-24); the remaining
-//      CTAs quantize one 128-row Q block each (Q does not depend on the mean,
-//      so its quantization overlaps the K reduction).
-//   2. kmean_finalize: sums the chunk partials in int64 (exact, order free)
-//      and writes the fp32 mean per (batch, kv head, channel).
-//   3. quant_k: smooths and quantizes one 64-row K block per CTA.
+// One launch, HBM-bound.  The grid is made of thread-block clusters of
+// kCluster CTAs (16 when there are few kv heads, so the K work still spreads
+// over the chip):
+//   * K clusters (one per batch and kv head): CTA r of the cluster owns a
+//     range of whole 64-row K blocks.  Pass 1 sums its rows per channel
+//     exactly (fp16 values accumulated in double, at most 2^13 terms per
+//     thread, then int64 counts of 2^-24); the cluster then adds the
+//     kCluster partial sums through distributed shared memory in a fixed
+//     order, so every CTA holds the same exact mean (rank 0 stores it).
+//     Pass 2 re-reads its rows (from L2), subtracts the mean and quantizes
+//     its 64-row blocks, two at a time.
+//   * Q clusters: every CTA quantizes one 128-row Q block (Q does not depend
+//     on the mean, so this overlaps the K work).
 //
-// Every load is a coalesced 16-byte vector (8 fp16); a block's rows stay in
-// registers between the abs-max reduction (warp shuffles, then shared memory
-// across the 8 warps) and the rounding pass, so each element is read from HBM
-// once per pass.  All float operations use explicit IEEE round-to-nearest
-// intrinsics so the int8 codes and scales are bit-reproducible.
+// Loads are coalesced 16-byte vectors (8 fp16) kept as raw registers; the
+// abs-max (warp shuffles, then shared memory across warps) and the rounding
+// pass both convert from them, so nothing is read twice within a block.  All
+// float operations use explicit IEEE round-to-nearest intrinsics, so the int8
+// codes and scales are bit-reproducible.
+#include <cooperative_groups.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -23,10 +29,12 @@
 
 #include "sage_internal.h"
 
+namespace cg = cooperative_groups;
+
 namespace sage {
 
 constexpr int kQuantThreads = 256;
-constexpr int kMeanChunk = 256;  // tokens per K-mean partial
+constexpr int kCluster = 8;  // CTAs per K head (16 when there are few heads)
 
 // ------------------------------------------------------------- helpers
 
@@ -43,21 +51,35 @@ __device__ __forceinline__ float block_absmax(float v, float* red) {
     if (lane == 0) red[8] = w;
   }
   __syncthreads();
-  return red[8];
+  const float a = red[8];
+  __syncthreads();  // red[] may be reused by the next block
+  return a;
+}
+
+// Abs-max of NB independent blocks at once (one value per block per thread).
+template <int NB>
+__device__ __forceinline__ void block_absmax_n(float (&v)[NB], float* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v[b] = fmaxf(v[b], __shfl_xor_sync(0xffffffffu, v[b], o));
+    if (lane == 0) red[b * 8 + warp] = v[b];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    float a = red[b * 8];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) a = fmaxf(a, red[b * 8 + w]);
+    v[b] = a;
+  }
+  __syncthreads();  // red[] may be reused by the next group of blocks
 }
 
 __device__ __forceinline__ int quant_one(float x, float r) {
-  int t = __float2int_rn(__fmul_rn(x, r));  // round half to even
+  const int t = __float2int_rn(__fmul_rn(x, r));  // round half to even
   return max(-127, min(127, t));
-}
-
-__device__ __forceinline__ uint2 quant_pack8(const float (&x)[8], float r) {
-  uint32_t lo = 0, hi = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
-#pragma unroll
-  for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
-  return make_uint2(lo, hi);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
@@ -70,42 +92,41 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
   }
 }
 
-// Quantizes one block of `rows` x D values (row-major, fp16) into int8 and
-// returns the block scale fl32(amax/127).  `mean` (K only) is subtracted per
-// channel first.  ROWS_MAX is 128 (Q) or 64 (K).
+// Smoothed (for K) fp32 values of one 16-byte vector.
+template <bool SMOOTH>
+__device__ __forceinline__ void values8(const uint4& raw, const float (&m)[8], float (&x)[8]) {
+  unpack8(raw, x);
+  if (SMOOTH) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m[e]);
+  }
+}
+
+// Quantizes one block of `rows` x D fp16 values (row-major) into int8 and
+// returns its scale fl32(amax/127).  For K, `m` holds this thread's 8
+// channel means (the same channels for every vector of the thread).
 template <int D, int ROWS_MAX, bool SMOOTH>
 __device__ __forceinline__ float quant_block(const __half* __restrict__ src, int8_t* __restrict__ dst,
-                                             int rows, const float* __restrict__ mean, float* red) {
-  constexpr int TPR = D / 8;                                // 16-byte vectors per row
-  constexpr int VPT = ROWS_MAX * TPR / kQuantThreads;       // vectors per thread
+                                             int rows, const float (&m)[8], float* red) {
+  constexpr int TPR = D / 8;                           // 16-byte vectors per row
+  constexpr int VPT = ROWS_MAX * TPR / kQuantThreads;  // vectors per thread
   static_assert(VPT >= 1 && kQuantThreads % TPR == 0, "bad block shape");
   const int nvec = rows * TPR;
   const int tid = threadIdx.x;
-
-  float m[8];
-  if (SMOOTH) {
-    const int ch0 = (tid % TPR) * 8;  // the same channels for every vector of this thread
-#pragma unroll
-    for (int e = 0; e < 8; ++e) m[e] = __ldg(mean + ch0 + e);
-  }
-
-  float x[VPT][8];
   uint4 raw[VPT];
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
     const int idx = tid + v * kQuantThreads;
-    raw[v] = idx < nvec ? __ldg(reinterpret_cast<const uint4*>(src) + idx) : make_uint4(0, 0, 0, 0);
+    raw[v] = idx < nvec ? __ldcs(reinterpret_cast<const uint4*>(src) + idx) : make_uint4(0, 0, 0, 0);
   }
   float amax = 0.f;
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
-    unpack8(raw[v], x[v]);
-    const bool live = tid + v * kQuantThreads < nvec;  // padding rows are not in the block
+    if (tid + v * kQuantThreads < nvec) {  // padding rows are not in the block
+      float x[8];
+      values8<SMOOTH>(raw[v], m, x);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float t = SMOOTH ? __fsub_rn(x[v][e], m[e]) : x[v][e];
-      x[v][e] = live ? t : 0.f;
-      amax = fmaxf(amax, fabsf(x[v][e]));
+      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
     }
   }
   const float a = block_absmax(amax, red);
@@ -113,119 +134,205 @@ __device__ __forceinline__ float quant_block(const __half* __restrict__ src, int
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
     const int idx = tid + v * kQuantThreads;
-    if (idx < nvec) reinterpret_cast<uint2*>(dst)[idx] = quant_pack8(x[v], r);
+    if (idx < nvec) {
+      float x[8];
+      values8<SMOOTH>(raw[v], m, x);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
+      __stcs(reinterpret_cast<uint2*>(dst) + idx, make_uint2(lo, hi));
+    }
   }
   return a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
 }
 
-// ------------------------------------------------------------- kernels
-
-// Exact column sums of one 256-token chunk of K for one (batch, kv head).
-// A thread sums at most kMeanChunk / RPP values per channel in double, which
-// is exact (fp16 values are multiples of 2^-24 below 2^16 in magnitude, and
-// the partial stays below 2^53 units); the result is an int64 count of 2^-24.
-template <int D>
-__device__ __forceinline__ void kmean_chunk(const __half* __restrict__ k, long long* __restrict__ part,
-                                            int Lk, int bhk, int chunk, int nchunks,
-                                            long long* red /* [RPP][D] */) {
+// Smooths and quantizes NB consecutive K blocks [kb, kb+NB) of one head
+// (rows beyond Lk are padding; blocks at or beyond kb_end are skipped).
+template <int D, int NB>
+__device__ __forceinline__ void quant_k_blocks(const __half* __restrict__ kh, int8_t* __restrict__ kq,
+                                               float* __restrict__ ks, int kb, int kb_end, int Lk,
+                                               const float (&m)[8], float* red) {
   constexpr int TPR = D / 8;
-  constexpr int RPP = kQuantThreads / TPR;  // rows per pass
+  constexpr int VPT = SAGE_K_BLOCK_ROWS * TPR / kQuantThreads;
   const int tid = threadIdx.x;
-  const int cg = tid % TPR, rr = tid / TPR;
-  const int t0 = chunk * kMeanChunk;
-  const int t1 = min(Lk, t0 + kMeanChunk);
-  const uint4* base = reinterpret_cast<const uint4*>(k + (size_t)bhk * Lk * D) + cg;
-  double acc[8];
+  uint4 raw[NB][VPT];
+  int nvec[NB];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-#pragma unroll 4
-  for (int t = t0 + rr; t < t1; t += RPP) {
-    float x[8];
-    unpack8(__ldg(base + (size_t)t * TPR), x);
+  for (int b = 0; b < NB; ++b) {
+    const int r0 = (kb + b) * SAGE_K_BLOCK_ROWS;
+    nvec[b] = kb + b < kb_end ? min(SAGE_K_BLOCK_ROWS, Lk - r0) * TPR : 0;
+    const uint4* src = reinterpret_cast<const uint4*>(kh + (size_t)r0 * D);
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] += (double)x[e];
+    for (int v = 0; v < VPT; ++v) {
+      const int idx = tid + v * kQuantThreads;
+      raw[b][v] = idx < nvec[b] ? __ldcs(src + idx) : make_uint4(0, 0, 0, 0);
+    }
   }
+  float amax[NB];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[rr * D + cg * 8 + e] = (long long)(acc[e] * 16777216.0);
-  __syncthreads();
-  for (int c = tid; c < D; c += kQuantThreads) {
-    long long s = 0;
-    for (int i = 0; i < RPP; ++i) s += red[i * D + c];
-    part[((size_t)bhk * nchunks + chunk) * D + c] = s;
+  for (int b = 0; b < NB; ++b) {
+    amax[b] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      if (tid + v * kQuantThreads < nvec[b]) {
+        float x[8];
+        values8<true>(raw[b][v], m, x);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax[b] = fmaxf(amax[b], fabsf(x[e]));
+      }
+    }
+  }
+  block_absmax_n<NB>(amax, red);
+#pragma unroll
+  for (int b = 0; b < NB; ++b) {
+    const float a = amax[b];
+    const float r = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+    uint2* dst = reinterpret_cast<uint2*>(kq + (size_t)(kb + b) * SAGE_K_BLOCK_ROWS * D);
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+      const int idx = tid + v * kQuantThreads;
+      if (idx < nvec[b]) {
+        float x[8];
+        values8<true>(raw[b][v], m, x);
+        uint32_t lo = 0, hi = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
+        __stcs(dst + idx, make_uint2(lo, hi));
+      }
+    }
+    if (tid == 0 && nvec[b] > 0) ks[kb + b] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
   }
 }
 
+// ------------------------------------------------------------- kernel
+
 template <int D>
 __global__ void __launch_bounds__(kQuantThreads)
-kmean_and_quant_q_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
-                         int8_t* __restrict__ q_i8, float* __restrict__ q_scale,
-                         long long* __restrict__ part, int BHkv, int BH, int Lq, int Lk,
-                         int nchunks, int nqb, float c) {
-  __shared__ float red[16];
-  __shared__ long long kred[kQuantThreads / (D / 8) * D];
-  const int n_mean = BHkv * nchunks;
-  int blk = blockIdx.x;
-  if (blk < n_mean) {
-    kmean_chunk<D>(k, part, Lk, blk / nchunks, blk % nchunks, nchunks, kred);
+quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
+                int8_t* __restrict__ q_i8, int8_t* __restrict__ k_i8,
+                float* __restrict__ q_scale, float* __restrict__ k_scale,
+                float* __restrict__ k_mean, int BHkv, int Lq, int Lk, int nqb, int nkb,
+                int kb_per_cta, int n_k_ctas, int n_q_blocks, float c) {
+  constexpr int TPR = D / 8;
+  constexpr int RPP = kQuantThreads / TPR;  // rows per pass of the column sums
+  __shared__ float red[32];
+  __shared__ long long part[D];   // this CTA's exact column sums (units of 2^-24)
+  __shared__ long long rsum[RPP * D > 0 ? RPP * D : 1];
+  __shared__ float mean[D];
+  const int tid = threadIdx.x;
+  const float no_mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+
+  if ((int)blockIdx.x >= n_k_ctas) {
+    // ------------------------------------------------------------ Q block
+    const int blk = blockIdx.x - n_k_ctas;
+    if (blk >= n_q_blocks) return;  // padding CTA of the last cluster
+    const int bh = blk / nqb, qb = blk - bh * nqb;
+    const int r0 = qb * SAGE_Q_BLOCK_ROWS;
+    const size_t off = ((size_t)bh * Lq + r0) * D;
+    const float s = quant_block<D, SAGE_Q_BLOCK_ROWS, false>(
+        q + off, q_i8 + off, min(SAGE_Q_BLOCK_ROWS, Lq - r0), no_mean, red);
+    if (tid == 0) q_scale[blk] = __fmul_rn(s, c);
     return;
   }
-  blk -= n_mean;
-  const int bh = blk / nqb, qb = blk - bh * nqb;
-  const int r0 = qb * SAGE_Q_BLOCK_ROWS;
-  const int rows = min(SAGE_Q_BLOCK_ROWS, Lq - r0);
-  const size_t off = ((size_t)bh * Lq + r0) * D;
-  const float s = quant_block<D, SAGE_Q_BLOCK_ROWS, false>(q + off, q_i8 + off, rows, nullptr, red);
-  if (threadIdx.x == 0) q_scale[blk] = __fmul_rn(s, c);
-}
 
-template <int D>
-__global__ void kmean_finalize_kernel(const long long* __restrict__ part, float* __restrict__ k_mean,
-                                      int Lk, int nchunks) {
-  const int bhk = blockIdx.x, c = threadIdx.x;
-  long long s = 0;
-  for (int i = 0; i < nchunks; ++i) s += part[((size_t)bhk * nchunks + i) * D + c];
-  const double mean = __ddiv_rn(__dmul_rn(__ll2double_rn(s), 0x1p-24), (double)Lk);
-  k_mean[(size_t)bhk * D + c] = __double2float_rn(mean);
-}
+  // -------------------------------------------------------------- K head
+  cg::cluster_group cluster = cg::this_cluster();
+  const int ncl = (int)cluster.num_blocks();
+  const int rank = (int)cluster.block_rank();
+  const int bhk = blockIdx.x / ncl;
+  const int kb0 = min(nkb, rank * kb_per_cta), kb1 = min(nkb, kb0 + kb_per_cta);
+  const int t0 = kb0 * SAGE_K_BLOCK_ROWS, t1 = min(Lk, kb1 * SAGE_K_BLOCK_ROWS);
+  const __half* kh = k + (size_t)bhk * Lk * D;
 
-template <int D>
-__global__ void __launch_bounds__(kQuantThreads)
-quant_k_kernel(const __half* __restrict__ k, const float* __restrict__ k_mean,
-               int8_t* __restrict__ k_i8, float* __restrict__ k_scale, int Lk, int nkb) {
-  __shared__ float red[16];
-  const int blk = blockIdx.x;
-  const int bhk = blk / nkb, kb = blk - bhk * nkb;
-  const int r0 = kb * SAGE_K_BLOCK_ROWS;
-  const int rows = min(SAGE_K_BLOCK_ROWS, Lk - r0);
-  const size_t off = ((size_t)bhk * Lk + r0) * D;
-  const float s = quant_block<D, SAGE_K_BLOCK_ROWS, true>(k + off, k_i8 + off, rows,
-                                                          k_mean + (size_t)bhk * D, red);
-  if (threadIdx.x == 0) k_scale[blk] = s;
+  // pass 1: exact column sums of rows [t0, t1)
+  {
+    const int cg8 = tid % TPR, rr = tid / TPR;
+    const uint4* base = reinterpret_cast<const uint4*>(kh) + cg8;
+    double acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.0;
+#pragma unroll 8
+    for (int t = t0 + rr; t < t1; t += RPP) {
+      float x[8];
+      unpack8(__ldg(base + (size_t)t * TPR), x);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += (double)x[e];
+    }
+    // fp16 values are multiples of 2^-24 below 2^16: each double sum of at
+    // most 2^13 of them is exact, and so is its conversion to int64
+#pragma unroll
+    for (int e = 0; e < 8; ++e) rsum[rr * D + cg8 * 8 + e] = (long long)(acc[e] * 16777216.0);
+    __syncthreads();
+    for (int ch = tid; ch < D; ch += kQuantThreads) {
+      long long s = 0;
+      for (int i = 0; i < RPP; ++i) s += rsum[i * D + ch];
+      part[ch] = s;
+    }
+  }
+  cluster.sync();  // every CTA's partial sums are visible cluster-wide
+  for (int ch = tid; ch < D; ch += kQuantThreads) {
+    long long s = 0;
+    for (int r = 0; r < ncl; ++r) s += *cluster.map_shared_rank(&part[ch], r);
+    const double mu = __ddiv_rn(__dmul_rn(__ll2double_rn(s), 0x1p-24), (double)Lk);
+    mean[ch] = __double2float_rn(mu);
+    if (rank == 0) k_mean[(size_t)bhk * D + ch] = mean[ch];
+  }
+  cluster.sync();  // no CTA leaves (or reuses part[]) while others read it
+
+  // pass 2: smooth and quantize this CTA's K blocks
+  float m8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) m8[e] = mean[(tid % TPR) * 8 + e];
+  for (int kb = kb0; kb < kb1; kb += 2)
+    quant_k_blocks<D, 2>(k + (size_t)bhk * Lk * D, k_i8 + (size_t)bhk * Lk * D,
+                         k_scale + (size_t)bhk * nkb, kb, kb1, Lk, m8, red);
 }
 
 // ------------------------------------------------------------- launcher
 
-size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d) {
-  const size_t nchunks = (size_t)(Lk + kMeanChunk - 1) / kMeanChunk;
-  return (size_t)B * Hkv * nchunks * d * sizeof(long long);
-}
+size_t quant_workspace_bytes(int, int, int, int) { return 0; }
 
 template <int D>
 static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* launches) {
   const int BH = a.B * a.H, BHkv = a.B * a.Hkv;
-  const int nchunks = (a.Lk + kMeanChunk - 1) / kMeanChunk;
   const int nqb = (a.Lq + SAGE_Q_BLOCK_ROWS - 1) / SAGE_Q_BLOCK_ROWS;
   const int nkb = (a.Lk + SAGE_K_BLOCK_ROWS - 1) / SAGE_K_BLOCK_ROWS;
-  long long* part = static_cast<long long*>(a.workspace);
-  const long long g1 = (long long)BHkv * nchunks + (long long)BH * nqb;
-  const long long g3 = (long long)BHkv * nkb;
-  if (g1 > 0x7fffffffLL || g3 > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kmean_and_quant_q_kernel<D><<<(unsigned)g1, kQuantThreads, 0, st>>>(
-      a.q, a.k, a.q_i8, a.q_scale, part, BHkv, BH, a.Lq, a.Lk, nchunks, nqb, a.c);
-  kmean_finalize_kernel<D><<<BHkv, D, 0, st>>>(part, a.k_mean, a.Lk, nchunks);
-  quant_k_kernel<D><<<(unsigned)g3, kQuantThreads, 0, st>>>(a.k, a.k_mean, a.k_i8, a.k_scale,
-                                                           a.Lk, nkb);
-  *launches += 3;
+  auto kern = quant_qk_kernel<D>;
+  // few heads: wider clusters so the K work spreads over more SMs
+  int cl = kCluster;
+  if ((long long)BHkv * kCluster < 256 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)
+    cl = 16;
+  const int kb_per_cta = (nkb + cl - 1) / cl;
+  // a CTA sums at most kb_per_cta * 64 rows; each thread at most 1/RPP of them
+  if ((long long)kb_per_cta * SAGE_K_BLOCK_ROWS / (kQuantThreads / (D / 8)) > 8192)
+    return cudaErrorInvalidValue;
+  const long long n_k_ctas = (long long)BHkv * cl;
+  const long long n_q_blocks = (long long)BH * nqb;
+  const long long n_q_ctas = (n_q_blocks + cl - 1) / cl * cl;
+  if (n_k_ctas + n_q_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(n_k_ctas + n_q_ctas), 1, 1);
+  cfg.blockDim = dim3(kQuantThreads, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cl;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a.q, a.k, a.q_i8, a.k_i8, a.q_scale, a.k_scale,
+                                     a.k_mean, BHkv, a.Lq, a.Lk, nqb, nkb, kb_per_cta,
+                                     (int)n_k_ctas, (int)n_q_blocks, a.c);
+  *launches += 1;
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

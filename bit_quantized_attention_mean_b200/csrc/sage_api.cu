@@ -106,12 +106,13 @@ sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* ws = workspace;
-  if (!ws && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  const bool own = !ws && need > 0;
+  if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
   sage::QuantArgs a{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
                     q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale)};
   int launches = 0;
   cudaError_t e = sage::launch_quant(a, s, &launches);
-  if (!workspace && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
   g_last_launches = launches;
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

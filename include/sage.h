@@ -74,7 +74,9 @@ typedef enum {
  *   k_mean   fp32 [B, Hkv, d]              (out) mean of K over all Lk tokens
  *   workspace, workspace_bytes: device scratch of at least
  *            sage_quant_workspace_size(B, Hkv, Lk, d) bytes, or NULL/0 to let
- *            the call allocate it with cudaMallocAsync on `stream`.
+ *            the call allocate it with cudaMallocAsync on `stream`.  The
+ *            current kernels need none (the size is 0; the K mean is reduced
+ *            in on-chip distributed shared memory), so NULL/0 is always fine.
  *
  * Per block: a = max|x|, r = fl32(127/a), q = clamp(rne(fl32(x*r)), -127, 127);
  * an all-zero block gives q = 0 and scale 0.  For K, x = fl32(float(K) - m),
@@ -88,7 +90,7 @@ SAGE_API sage_status sage_quant_qk(const void *q, const void *k,
                           float sm_scale, void *workspace, size_t workspace_bytes,
                           void *stream);
 
-/* Bytes of scratch sage_quant_qk needs (exact int64 partial sums of K). */
+/* Bytes of scratch sage_quant_qk needs (currently 0). */
 SAGE_API size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d);
 
 /*
