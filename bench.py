@@ -50,8 +50,8 @@ INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (sha256 of attn.cu); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "af67746c1937cbdf", "workload": "llm-causal-B1H32L4096d128",
-               "bytes_per_launch": 67173888 + 6658048}
+NCU_TRAFFIC = {"attn_sha": "f280fd201cc6af7f", "workload": "llm-causal-B1H32L4096d128",
+               "bytes_per_launch": 68573184 + 7489792}
 
 
 def load_peaks():
@@ -371,7 +371,7 @@ def run_ours(args, w):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))

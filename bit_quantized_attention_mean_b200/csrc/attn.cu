@@ -48,6 +48,7 @@ namespace sage {
 
 __device__ int g_device_status;
 
+constexpr long long kGlobalOrderKVBytes = 112ll << 20;  // K/V total that stays L2-resident
 constexpr int BQ = 128;  // query rows per tile  (= Q quantization block)
 constexpr int BK = 64;   // key rows per tile    (= K quantization block)
 
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(192, 2)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                      const float* __restrict__ k_scale, __half* __restrict__ out, int H, int Hkv,
-                     int Lq, int Lk, int nqt) {
+                     int Lq, int Lk, int nqt, int global_lpt) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment of the shared-window address (swizzle atoms)
@@ -109,9 +110,19 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int bh = blockIdx.x / nqt;
-  int qt = blockIdx.x - bh * nqt;
-  if (CAUSAL) qt = nqt - 1 - qt;  // longest rows first within a head
+  // Causal tiles differ in length; launch the longest first.  When the K/V
+  // of every head fit in L2 together, order across heads (global longest
+  // first); otherwise keep each head's tiles together so its K/V stay hot.
+  int bh, qt;
+  if (CAUSAL && global_lpt) {
+    const int BH = gridDim.x / nqt;
+    qt = nqt - 1 - (int)(blockIdx.x / BH);
+    bh = blockIdx.x - (nqt - 1 - qt) * BH;
+  } else {
+    bh = blockIdx.x / nqt;
+    qt = blockIdx.x - bh * nqt;
+    if (CAUSAL) qt = nqt - 1 - qt;  // longest rows first within a head
+  }
   const int h = bh % H, b = bh / H;
   const int bhk = b * Hkv + h / (H / Hkv);
   const int q0 = qt * BQ;
@@ -303,9 +314,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       float lsum = 0.f;
 #pragma unroll
       for (int k = 0; k < BK; k += 2) {
-        // exact int -> float: reinterpret (S + 1.5*2^23) and subtract 1.5*2^23
-        const float x0 = __fsub_rn(__int_as_float((int)s[k] + 0x4B400000), 12582912.f);
-        const float x1 = __fsub_rn(__int_as_float((int)s[k + 1] + 0x4B400000), 12582912.f);
+        // |S| <= 127*127*128 < 2^24: the int -> float conversion is exact
+        const float x0 = __int2float_rn((int)s[k]);
+        const float x1 = __int2float_rn((int)s[k + 1]);
         float p0 = ex2_approx(fmaf(x0, c, -moff));
         float p1 = ex2_approx(fmaf(x1, c, -moff));
         if (!full) {
@@ -412,9 +423,11 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launch
 
   const int nqt = (a.Lq + BQ - 1) / BQ;
   const long long grid = (long long)a.B * a.H * nqt;
+  const long long kv_bytes = (long long)a.B * a.Hkv * a.Lk * D * 3;  // int8 K + fp16 V
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.out, a.H,
-                                                   a.Hkv, a.Lq, a.Lk, nqt);
+                                                   a.Hkv, a.Lq, a.Lk, nqt,
+                                                   kv_bytes <= kGlobalOrderKVBytes ? 1 : 0);
   *launches += 1;
   return cudaGetLastError();
 }
