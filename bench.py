@@ -49,8 +49,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"
 INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
-# kernel source it was taken on (sha256 of attn.cu); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "f280fd201cc6af7f", "workload": "llm-causal-B1H32L4096d128",
+# kernel source it was taken on (attn_source_hash); otherwise reported null.
+NCU_TRAFFIC = {"attn_sha": "4db0ac417f080078", "workload": "llm-causal-B1H32L4096d128",
                "bytes_per_launch": 68573184 + 7489792}
 
 
@@ -65,9 +65,16 @@ def load_peaks():
 
 
 def attn_source_hash():
-    p = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc", "attn.cu")
-    with open(p, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """Hash of the attention kernel's device code (attn.cu up to its host
+    section) and of the PTX wrappers it is built from."""
+    csrc = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc")
+    with open(os.path.join(csrc, "attn.cu"), "rb") as f:
+        text = f.read()
+    marker = b"// ------------------------------------------------------------------- host"
+    h = hashlib.sha256(text.split(marker)[0])
+    with open(os.path.join(csrc, "sm100_ptx.cuh"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 # ------------------------------------------------------------ clock sampler
@@ -149,6 +156,28 @@ def dist_setup():
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
     return world, rank, local
+
+
+def aggregate_over_ranks(times_ms, launches, world, device):
+    """Job-level numbers from per-rank ones: every time is the maximum over
+    ranks (the slowest GPU sets the job's pace), the launch count is the sum.
+    Works on any initialized torch.distributed backend (NCCL on GPUs, gloo
+    on CPU); with world == 1 it returns the inputs unchanged."""
+    import torch
+    if world <= 1:
+        return list(times_ms), int(launches)
+    import torch.distributed as dist
+    t = torch.tensor(list(times_ms), dtype=torch.float64, device=device)
+    n = torch.tensor([int(launches)], dtype=torch.int64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return t.tolist(), int(n.item())
+
+
+def weak_scaling_value(ops_per_rank, world, ms_per_step):
+    """Whole-job throughput in TOPS: every rank does ops_per_rank per step and
+    a step takes ms_per_step (the maximum over ranks)."""
+    return world * ops_per_rank / (ms_per_step * 1e-3) / 1e12
 
 
 # ------------------------------------------------------------ CPU oracle
@@ -304,19 +333,14 @@ def run_ours(args, w):
     sage.sage_check_device_status(stream)
     e2e_ms = float(sum(a.elapsed_time(b) for a, b in e2e_ev) / e2e_steps)
 
-    stats = torch.tensor([total_ms, attn_avg_ms, e2e_ms, quant_avg_ms], dtype=torch.float64,
-                         device=dev)
-    nl = torch.tensor([launches], dtype=torch.int64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(stats, op=torch.distributed.ReduceOp.MAX)
-        torch.distributed.all_reduce(nl, op=torch.distributed.ReduceOp.SUM)
-    total_ms, attn_avg_ms, e2e_ms, quant_avg_ms = stats.tolist()
+    (total_ms, attn_avg_ms, e2e_ms, quant_avg_ms), n_launches = aggregate_over_ranks(
+        [total_ms, attn_avg_ms, e2e_ms, quant_avg_ms], launches, world, dev)
 
     result = None
     if rank == 0:
         ops = 4.0 * d * w.pairs()
         ms_per_step = total_ms / n
-        value = world * ops / (ms_per_step * 1e-3) / 1e12
+        value = weak_scaling_value(ops, world, ms_per_step)
         peaks = load_peaks()
         p16 = float(peaks["bf16_tflops"])
         p8 = INT8_OVER_FP16 * p16
@@ -344,10 +368,10 @@ def run_ours(args, w):
                                        f"{INT8_OVER_FP16} x P_fp16 (nominal ratio)")},
             "kernel_ms": {"attention": attn_avg_ms, "quant": quant_avg_ms},
             "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
-            "e2e": {"value": world * ops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+            "e2e": {"value": weak_scaling_value(ops, world, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": int(qn.nbytes + kn.nbytes + vn.nbytes),
                     "d2h_bytes_per_step": int(qn.nbytes)},
-            "gpu_launches": int(nl.item()),
+            "gpu_launches": n_launches,
             "clocks": clocks.summary(),
         }
     if world > 1:

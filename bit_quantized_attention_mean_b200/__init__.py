@@ -26,6 +26,7 @@ from ._lib import (  # noqa: F401
     sage_attn_fwd_prequant,
     sage_attn_workspace_size,
     sage_check_device_status,
+    sage_debug_wait_timeout,
     sage_last_launch_count,
     sage_quant_qk,
     sage_quant_workspace_size,

@@ -27,6 +27,7 @@ SYMBOLS = (
     "sage_status_string",
     "sage_last_launch_count",
     "sage_attn_fwd_noalloc",
+    "sage_debug_wait_timeout",
 )
 
 STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
@@ -73,6 +74,8 @@ def load_library():
         lib.sage_status_string.restype = ctypes.c_char_p
         lib.sage_attn_fwd_noalloc.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
         lib.sage_attn_fwd_noalloc.restype = I
+        lib.sage_debug_wait_timeout.argtypes = [I, P]
+        lib.sage_debug_wait_timeout.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -223,6 +226,13 @@ def sage_attn_fwd_host(q, k, v, out, causal, sm_scale, stream=None):
         ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
         B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
         "sage_attn_fwd_host")
+
+
+def sage_debug_wait_timeout(limit_ms, stream=None):
+    """Launch the diagnostic kernel whose bounded wait must give up after
+    limit_ms; the next sage_check_device_status then raises SAGE_ERR_TIMEOUT."""
+    _check(load_library().sage_debug_wait_timeout(int(limit_ms), _stream(stream)),
+           "sage_debug_wait_timeout")
 
 
 def sage_check_device_status(stream=None):

@@ -90,8 +90,8 @@ struct AttnCfg {
 
 // Warp-uniform bounded wait: every lane waits, then the warp agrees.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int site) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, &g_device_status, site);
+                                          int site, uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, &g_device_status, site, limit_ns);
   return __all_sync(0xffffffffu, ok);
 }
 
@@ -438,6 +438,26 @@ cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches) {
                     : launch_attn_t<128, false>(a, st, launches);
   return a.causal ? launch_attn_t<64, true>(a, st, launches)
                   : launch_attn_t<64, false>(a, st, launches);
+}
+
+// One warp waits on an mbarrier that nothing ever completes, through the
+// same bounded wait the attention kernel uses; after limit_ns the wait gives
+// up, raises the CTA's abort flag and records site 99 in the status word.
+__global__ void bounded_wait_probe_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  __syncwarp();
+  warp_wait(&bar, 0, &abort_flag, 99, limit_ns);
+}
+
+cudaError_t launch_wait_probe(int limit_ms, cudaStream_t st) {
+  bounded_wait_probe_kernel<<<1, 32, 0, st>>>((uint64_t)limit_ms * 1000000ull);
+  return cudaGetLastError();
 }
 
 cudaError_t read_and_clear_device_status(int* value) {

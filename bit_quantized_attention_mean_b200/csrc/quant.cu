@@ -77,8 +77,15 @@ __device__ __forceinline__ void block_absmax_n(float (&v)[NB], float* red) {
   __syncthreads();  // red[] may be reused by the next group of blocks
 }
 
+// rne(fl32(x * r)) clamped to [-127, 127], as an int.  The rounding adds
+// 1.5 * 2^23 in fp32 (the FADD itself rounds to the nearest integer, ties to
+// even, exactly as cvt.rni would for |x * r| < 2^22) and reads the integer
+// back from the low mantissa bits; this keeps the conversion off the
+// transcendental/conversion unit.
 __device__ __forceinline__ int quant_one(float x, float r) {
-  const int t = __float2int_rn(__fmul_rn(x, r));  // round half to even
+  const float y = __fmul_rn(x, r);
+  const float big = __fadd_rn(y, 12582912.f);
+  const int t = __float_as_int(big) - 0x4B400000;
   return max(-127, min(127, t));
 }
 

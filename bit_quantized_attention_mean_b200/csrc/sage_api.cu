@@ -211,6 +211,15 @@ sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const voi
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
+sage_status sage_debug_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 2000) return SAGE_ERR_INVALID_ARG;
+  sage_status st = check_device();
+  if (st != SAGE_OK) return st;
+  return sage::launch_wait_probe(limit_ms, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SAGE_OK
+             : SAGE_ERR_CUDA;
+}
+
 sage_status sage_check_device_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGE_ERR_CUDA;
   int v = 0;

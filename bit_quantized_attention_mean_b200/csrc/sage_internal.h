@@ -44,6 +44,10 @@ size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d);
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st, int* launches);
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches);
 
+// Launches a one-warp kernel whose bounded wait can never be satisfied and
+// gives up after limit_ms (exercises the error path without a fault).
+cudaError_t launch_wait_probe(int limit_ms, cudaStream_t st);
+
 // Device status word written by kernels whose bounded waits gave up.
 cudaError_t read_and_clear_device_status(int* value);
 

@@ -166,6 +166,17 @@ SAGE_API size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, 
  */
 SAGE_API sage_status sage_check_device_status(void *stream);
 
+/*
+ * sage_debug_wait_timeout -- diagnostic with no counterpart in the article:
+ * launches on `stream` a one-warp kernel that waits, through the same bounded
+ * wait the attention kernel uses, on a barrier that nothing ever completes.
+ * After limit_ms (1..2000) the wait gives up and records the event, so the
+ * next sage_check_device_status(stream) returns SAGE_ERR_TIMEOUT (and clears
+ * it).  Used to test the error path without faulting or hanging the GPU.
+ * Returns SAGE_ERR_INVALID_ARG for limit_ms outside 1..2000.
+ */
+SAGE_API sage_status sage_debug_wait_timeout(int limit_ms, void *stream);
+
 /* Static, human-readable name of a status code. */
 SAGE_API const char *sage_status_string(sage_status s);
 
