@@ -65,6 +65,11 @@ def _load():
         lib.oracle_quant_qk.restype = None
         lib.oracle_attn_quant_sim.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, P, I64, P]
         lib.oracle_attn_quant_sim.restype = None
+        lib.oracle_quant_qk_blocks.argtypes = [P, P, I, I, I, I, I, I, D, I, I, P, P, P, P, P]
+        lib.oracle_quant_qk_blocks.restype = None
+        lib.oracle_attn_quant_sim_blocks.argtypes = [P, P, P, P, P, I, I, I, I, I, I, I, I, P,
+                                                     I64, P]
+        lib.oracle_attn_quant_sim_blocks.restype = None
         lib.oracle_attn_fp64.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P, I64, P]
         lib.oracle_attn_fp64.restype = None
         lib.oracle_num_threads.argtypes = []
@@ -105,26 +110,30 @@ def k_mean(k: np.ndarray) -> np.ndarray:
     return out
 
 
-def quant_qk(q: np.ndarray, k: np.ndarray, sm_scale: float, smooth: bool = True):
-    """Returns (q_i8, k_i8, q_scale, k_scale, k_mean) as numpy arrays."""
+def quant_qk(q: np.ndarray, k: np.ndarray, sm_scale: float, smooth: bool = True,
+             q_block_rows: int = 128):
+    """Returns (q_i8, k_i8, q_scale, k_scale, k_mean) as numpy arrays.
+    q_block_rows: rows per Q quantization block (128 = the attention tile,
+    1 = one scale per query token)."""
     q = _c(q, np.float16)
     k = _c(k, np.float16)
     B, H, Lq, d = q.shape
     Bk, Hkv, Lk, dk = k.shape
     assert Bk == B and dk == d
-    nqb, nkb = -(-Lq // 128), -(-Lk // 64)
+    nqb, nkb = -(-Lq // q_block_rows), -(-Lk // 64)
     q_i8 = np.empty(q.shape, dtype=np.int8)
     k_i8 = np.empty(k.shape, dtype=np.int8)
     q_scale = np.empty((B, H, nqb), dtype=np.float32)
     k_scale = np.empty((B, Hkv, nkb), dtype=np.float32)
     km = np.empty((B, Hkv, d), dtype=np.float32)
-    _load().oracle_quant_qk(_ptr(q), _ptr(k), B, H, Hkv, Lq, Lk, d, float(sm_scale),
-                            1 if smooth else 0, _ptr(q_i8), _ptr(k_i8), _ptr(q_scale),
-                            _ptr(k_scale), _ptr(km))
+    _load().oracle_quant_qk_blocks(_ptr(q), _ptr(k), B, H, Hkv, Lq, Lk, d, float(sm_scale),
+                                   1 if smooth else 0, int(q_block_rows), _ptr(q_i8),
+                                   _ptr(k_i8), _ptr(q_scale), _ptr(k_scale), _ptr(km))
     return q_i8, k_i8, q_scale, k_scale, km
 
 
-def attn_quant_sim(q_i8, k_i8, q_scale, k_scale, v, causal: bool, rows=None):
+def attn_quant_sim(q_i8, k_i8, q_scale, k_scale, v, causal: bool, rows=None,
+                   q_block_rows: int = 128):
     """Simulated quantized attention; returns float64 [n_rows, d]
     (or [B, H, Lq, d] when rows is None)."""
     q_i8 = _c(q_i8, np.int8)
@@ -141,9 +150,10 @@ def attn_quant_sim(q_i8, k_i8, q_scale, k_scale, v, causal: bool, rows=None):
         rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
         out = np.empty((rows.shape[0], d), dtype=np.float64)
         rp, n = _ptr(rows), rows.shape[0]
-    _load().oracle_attn_quant_sim(_ptr(q_i8), _ptr(k_i8), _ptr(q_scale), _ptr(k_scale),
-                                  _ptr(v), B, H, Hkv, Lq, Lk, d, 1 if causal else 0,
-                                  rp, n, _ptr(out))
+    _load().oracle_attn_quant_sim_blocks(_ptr(q_i8), _ptr(k_i8), _ptr(q_scale),
+                                         _ptr(k_scale), _ptr(v), B, H, Hkv, Lq, Lk, d,
+                                         1 if causal else 0, int(q_block_rows), rp, n,
+                                         _ptr(out))
     return out
 
 

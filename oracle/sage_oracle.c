@@ -142,12 +142,28 @@ static float quant_block(const float *x, int rows, int d, int8_t *q)
  *   k  fp16 [B, Hkv, Lk, d]   -> k_i8 [B, Hkv, Lk, d], k_scale [B, Hkv, ceil(Lk/64)]
  *   k_mean [B, Hkv, d]        (written)
  * smooth = 0 skips the mean subtraction (ablation only; k_mean is then 0). */
+void oracle_quant_qk_blocks(const uint16_t *q, const uint16_t *k, int B, int H, int Hkv,
+                            int Lq, int Lk, int d, double sm_scale, int smooth,
+                            int BQ, int8_t *q_i8, int8_t *k_i8, float *q_scale,
+                            float *k_scale, float *k_mean);
+
 void oracle_quant_qk(const uint16_t *q, const uint16_t *k, int B, int H, int Hkv,
                      int Lq, int Lk, int d, double sm_scale, int smooth,
                      int8_t *q_i8, int8_t *k_i8, float *q_scale, float *k_scale,
                      float *k_mean)
 {
-    const int BQ = 128, BK = 64;
+    oracle_quant_qk_blocks(q, k, B, H, Hkv, Lq, Lk, d, sm_scale, smooth, 128, q_i8, k_i8,
+                           q_scale, k_scale, k_mean);
+}
+
+/* Same with Q blocks of BQ rows (1 = one scale per query token); K blocks
+ * stay 64 rows.  q_scale is [B, H, ceil(Lq / BQ)]. */
+void oracle_quant_qk_blocks(const uint16_t *q, const uint16_t *k, int B, int H, int Hkv,
+                            int Lq, int Lk, int d, double sm_scale, int smooth,
+                            int BQ, int8_t *q_i8, int8_t *k_i8, float *q_scale,
+                            float *k_scale, float *k_mean)
+{
+    const int BK = 64;
     const int nqb = (Lq + BQ - 1) / BQ, nkb = (Lk + BK - 1) / BK;
     const float c = (float)(sm_scale * 1.4426950408889634074);   /* log2(e) */
 
@@ -156,7 +172,7 @@ void oracle_quant_qk(const uint16_t *q, const uint16_t *k, int B, int H, int Hkv
     else
         for (int i = 0; i < B * Hkv * d; ++i) k_mean[i] = 0.0f;
 
-    float *buf = (float *)malloc(sizeof(float) * (size_t)BQ * d);
+    float *buf = (float *)malloc(sizeof(float) * (size_t)(BQ > BK ? BQ : BK) * d);
     for (int bh = 0; bh < B * H; ++bh) {
         for (int blk = 0; blk < nqb; ++blk) {
             int r0 = blk * BQ, rows = Lq - r0 < BQ ? Lq - r0 : BQ;
@@ -199,13 +215,30 @@ static int64_t visible_keys(int i, int Lq, int Lk, int causal)
  * in base-2 units), p = fp16(exp2(s - max s)), O = sum p v / sum p in fp64.
  * rows: flat indices (b*H + h)*Lq + i to compute, or NULL for all rows.
  * out: [n_rows, d] doubles (unrounded output). */
+void oracle_attn_quant_sim_blocks(const int8_t *q_i8, const int8_t *k_i8,
+                                  const float *q_scale, const float *k_scale,
+                                  const uint16_t *v, int B, int H, int Hkv, int Lq, int Lk,
+                                  int d, int causal, int BQ, const int64_t *rows,
+                                  int64_t n_rows, double *out);
+
 void oracle_attn_quant_sim(const int8_t *q_i8, const int8_t *k_i8,
                            const float *q_scale, const float *k_scale,
                            const uint16_t *v, int B, int H, int Hkv, int Lq, int Lk,
                            int d, int causal, const int64_t *rows, int64_t n_rows,
                            double *out)
 {
-    const int nqb = (Lq + 127) / 128, nkb = (Lk + 63) / 64;
+    oracle_attn_quant_sim_blocks(q_i8, k_i8, q_scale, k_scale, v, B, H, Hkv, Lq, Lk, d, causal,
+                                 128, rows, n_rows, out);
+}
+
+/* Same for q_scale blocks of BQ rows. */
+void oracle_attn_quant_sim_blocks(const int8_t *q_i8, const int8_t *k_i8,
+                                  const float *q_scale, const float *k_scale,
+                                  const uint16_t *v, int B, int H, int Hkv, int Lq, int Lk,
+                                  int d, int causal, int BQ, const int64_t *rows,
+                                  int64_t n_rows, double *out)
+{
+    const int nqb = (Lq + BQ - 1) / BQ, nkb = (Lk + 63) / 64;
     const int group = H / Hkv;
     if (!rows)
         n_rows = (int64_t)B * H * Lq;
@@ -226,7 +259,7 @@ void oracle_attn_quant_sim(const int8_t *q_i8, const int8_t *k_i8,
             if (nvis == 0)
                 continue;
             const int8_t *qi = q_i8 + (bh * Lq + i) * d;
-            double sq = (double)q_scale[bh * nqb + i / 128];
+            double sq = (double)q_scale[bh * nqb + i / BQ];
             double mx = -INFINITY;
             for (int64_t j = 0; j < nvis; ++j) {
                 const int8_t *kj = k_i8 + (bhk * Lk + j) * d;

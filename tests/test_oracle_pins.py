@@ -197,6 +197,53 @@ def test_quant_blocks_are_independent():
     assert got[2][0, 0, 1] == base[2][0, 0, 1]
 
 
+@pytest.mark.parametrize("bq", [64, 32, 1])
+def test_quant_properties_finer_q_blocks(bq):
+    """Q blocks of bq rows obey the same per-block definition: the largest
+    code of a non-zero block is 127, codes round x*127/amax to the nearest
+    integer, and the scale is amax/127 times c; K does not depend on bq."""
+    q, k, v = inputs.make_custom(1, 2, 2, 300, 200, 64, seed=5, k_offset_sigma=4.0)
+    sm = 1 / 8
+    q_i8, k_i8, q_scale, k_scale, km = oracle.quant_qk(q, k, sm, q_block_rows=bq)
+    c = np.float32(sm * math.log2(math.e))
+    assert q_scale.shape == (1, 2, -(-300 // bq))
+    for h in range(2):
+        for bi, (s, e) in enumerate(_blocks(300, bq)):
+            x = q[0, h, s:e].astype(np.float64)
+            qq = q_i8[0, h, s:e].astype(np.int32)
+            a = np.abs(x).max()
+            assert np.abs(qq).max() == 127
+            assert np.all(np.abs(qq - x * 127.0 / a) <= 0.5 + 1e-4)
+            assert abs(q_scale[0, h, bi] / c - a / 127) <= 2e-7 * a
+    base = oracle.quant_qk(q, k, sm)
+    for got, ref in zip((k_i8, k_scale, km), (base[1], base[3], base[4])):
+        assert np.array_equal(got, ref)
+
+
+def test_q_block_rows_one_is_per_token():
+    """With one-row blocks, scaling one token by a power of two changes only
+    that token's scale (its codes stay), and every other token is untouched;
+    a 32-row block that contains it changes its codes elsewhere in the block."""
+    q, k, v = inputs.make_custom(1, 1, 1, 96, 64, 64, seed=8)
+    base = oracle.quant_qk(q, k, 0.125, q_block_rows=1)
+    q2 = q.copy()
+    q2[0, 0, 40] *= np.float16(4)
+    got = oracle.quant_qk(q2, k, 0.125, q_block_rows=1)
+    assert np.array_equal(got[0], base[0])
+    assert got[2][0, 0, 40] == base[2][0, 0, 40] * np.float32(4)
+    keep = np.arange(96) != 40
+    assert np.array_equal(got[2][0, 0, keep], base[2][0, 0, keep])
+    b32 = oracle.quant_qk(q, k, 0.125, q_block_rows=32)
+    g32 = oracle.quant_qk(q2, k, 0.125, q_block_rows=32)
+    assert not np.array_equal(g32[0][0, 0, 32:64], b32[0][0, 0, 32:64])
+    assert np.array_equal(g32[0][0, 0, :32], b32[0][0, 0, :32])
+    assert np.array_equal(g32[0][0, 0, 64:], b32[0][0, 0, 64:])
+    # a single-token block is the whole tensor of that one token
+    one = oracle.quant_qk(np.ascontiguousarray(q[:, :, 40:41]), k, 0.125)
+    assert np.array_equal(one[0][0, 0, 0], base[0][0, 0, 40])
+    assert one[2][0, 0, 0] == base[2][0, 0, 40]
+
+
 def test_k_integer_shift_leaves_k_quant_unchanged():
     rng = np.random.default_rng(12)
     k = rng.integers(-30, 30, size=(1, 1, 128, 16)).astype(np.float16)
@@ -301,6 +348,41 @@ def test_sim_exact_quantization_reduces_to_fp64_attention():
     # and it is not the natural-exponent softmax (log2 e fold present)
     wrong = numpy_attention(q, k, v, True, float(np.float32(sm)) / math.log(2))
     assert np.max(np.abs(out - wrong)) > 1e-2
+
+
+def test_sim_per_token_scales_are_exact_where_tile_scales_are_not():
+    """Q rows that are 127-bounded integer vectors times a per-row power of
+    two quantize without error at one scale per token, so the simulation
+    then equals fp64 attention up to the fp16 rounding of P; one scale per
+    128-row tile rounds the small rows coarsely and misses that bound.  This
+    pins the row -> scale index of the simulation for every block height."""
+    rng = np.random.default_rng(77)
+    B, H, L, d = 1, 1, 256, 64
+    q = rng.integers(-127, 128, size=(B, H, L, d)).astype(np.float64)
+    q[..., 0] = 127
+    q *= 2.0 ** rng.integers(-6, 1, size=(B, H, L, 1))
+    half = rng.integers(-8, 9, size=(B, H, L // 2, d)).astype(np.float64)
+    half[:, :, ::32, 1] = 127
+    k = np.empty((B, H, L, d))
+    k[:, :, 0::2] = half
+    k[:, :, 1::2] = -half
+    v = rng.standard_normal((B, H, L, d))
+    q, k, v = (t.astype(np.float16) for t in (q, k, v))
+    sm = 1 / 512
+    ref = numpy_attention(q, k, v, False, float(np.float32(sm)))
+    bound = 2.0 ** -10 * np.abs(v.astype(np.float64)).max()
+    qk1 = oracle.quant_qk(q, k, sm, q_block_rows=1)
+    assert np.array_equal(qk1[0].astype(np.float64) * (qk1[2][..., None] /
+                          np.float32(sm * math.log2(math.e))).astype(np.float64),
+                          q.astype(np.float64))
+    out1 = oracle.attn_quant_sim(qk1[0], qk1[1], qk1[2], qk1[3], v, False, q_block_rows=1)
+    assert np.max(np.abs(out1 - ref)) < bound
+    qk128 = oracle.quant_qk(q, k, sm)
+    out128 = oracle.attn_quant_sim(qk128[0], qk128[1], qk128[2], qk128[3], v, False)
+    assert np.max(np.abs(out128 - ref)) > 4 * bound
+    # reading the per-token scales as if they were per-tile ones is wrong
+    wrong = oracle.attn_quant_sim(qk1[0], qk1[1], qk1[2][..., :2].copy(), qk1[3], v, False)
+    assert np.max(np.abs(wrong - ref)) > 4 * bound
 
 
 @pytest.mark.parametrize("causal", [False, True])
