@@ -1,7 +1,7 @@
 """Benchmark of the 8-bit quantized attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 1..5]
+                    [--workload 1..5] [--q-block-rows 128|64|32|1]
 
 A step is one pass of the whole hot path over the workload: K mean + Q/K
 quantization (sage_quant_qk) and the fused attention kernel
@@ -13,7 +13,9 @@ write) before every timed step, outside the step's CUDA events.
 Metric: TOPS = 4 * d * (unmasked query/key pairs) / step time, the QK^T and
 PV work counted at 2*d each.  ``e2e`` is the same metric through the public
 host-buffer call (sage_attn_fwd_host: H2D of q/k/v, forward pass, D2H of the
-output, all inside the timed region).  ``roofline`` reports the attention
+output, all inside the timed region).  ``--q-block-rows`` quantizes Q in
+blocks finer than the 128-row attention tile (the _qblock entry points; e2e
+then issues the same copies around sage_attn_fwd_qblock).  ``roofline`` reports the attention
 kernel against the combined tensor roofline: QK at the INT8 peak and PV at the
 FP16 peak, t_roof = 2*d*pairs/P_int8 + 2*d*pairs/P_fp16, with P_fp16 the
 measured bf16 peak and P_int8 = 2 x P_fp16 (nominal dense ratio).
@@ -182,18 +184,18 @@ def weak_scaling_value(ops_per_rank, world, ms_per_step):
 
 # ------------------------------------------------------------ CPU oracle
 
-def time_oracle_sample(w, q, k, v, n_rows, seed):
+def time_oracle_sample(w, q, k, v, n_rows, seed, qbr=128):
     """Oracle on a bounded sample: full Q/K quantization + n_rows query rows
     of the quantized-path simulation.  Returns (est_full_seconds, info)."""
     import oracle
     sm = float(np.float32(w.sm_scale))
     t0 = time.perf_counter()
-    qk = oracle.quant_qk(q, k, sm)
+    qk = oracle.quant_qk(q, k, sm, q_block_rows=qbr)
     t_quant = time.perf_counter() - t0
     rng = np.random.default_rng(seed)
     rows = np.sort(rng.choice(w.B * w.H * w.Lq, size=n_rows, replace=False)).astype(np.int64)
     t0 = time.perf_counter()
-    oracle.attn_quant_sim(*qk[:4], v, w.causal, rows=rows)
+    oracle.attn_quant_sim(*qk[:4], v, w.causal, rows=rows, q_block_rows=qbr)
     t_attn = time.perf_counter() - t0
     i = rows % w.Lq
     vis = np.minimum(w.Lk, np.maximum(0, i + (w.Lk - w.Lq) + 1)) if w.causal else np.full(n_rows, w.Lk)
@@ -213,7 +215,7 @@ def run_reference(args, w):
     times = []
     info = None
     for step in range(args.warmup + args.steps):
-        est, info = time_oracle_sample(w, q, k, v, rows, seed=step)
+        est, info = time_oracle_sample(w, q, k, v, rows, seed=step, qbr=args.q_block_rows)
         if step >= args.warmup:
             times.append(est)
     t = float(np.mean(times))
@@ -227,7 +229,7 @@ def run_reference(args, w):
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (int8 codes, int32 dot products)",
         "data": "synthetic (seeded numpy, fp16)",
-        "config": dict(w.describe(), l2="n/a (CPU)"),
+        "config": dict(w.describe(), q_block_rows=args.q_block_rows, l2="n/a (CPU)"),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": info["cores"],
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
@@ -264,7 +266,8 @@ def run_ours(args, w):
     B, H, Hkv, Lq, Lk, d = w.B, w.H, w.Hkv, w.Lq, w.Lk, w.d
     q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
     k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
-    q_scale = torch.empty((B, H, -(-Lq // 128)), dtype=torch.float32, device=dev)
+    qbr = args.q_block_rows
+    q_scale = torch.empty((B, H, -(-Lq // qbr)), dtype=torch.float32, device=dev)
     k_scale = torch.empty((B, Hkv, -(-Lk // 64)), dtype=torch.float32, device=dev)
     k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
     ws = torch.empty(max(1, sage.sage_quant_workspace_size(B, Hkv, Lk, d)), dtype=torch.uint8,
@@ -275,13 +278,21 @@ def run_ours(args, w):
 
     def step():
         nonlocal launches
-        sage.sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, workspace=ws,
-                           stream=stream)
+        if qbr == 128:
+            sage.sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, workspace=ws,
+                               stream=stream)
+        else:
+            sage.sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, qbr,
+                                      workspace=ws, stream=stream)
         launches += sage.sage_last_launch_count()
         ev_mid = torch.cuda.Event(enable_timing=True)
         ev_mid.record(stream)
-        sage.sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, w.causal,
-                                    stream=stream)
+        if qbr == 128:
+            sage.sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, w.causal,
+                                        stream=stream)
+        else:
+            sage.sage_attn_fwd_prequant_qblock(q_i8, k_i8, q_scale, k_scale, v, out, w.causal,
+                                               qbr, stream=stream)
         launches += sage.sage_last_launch_count()
         return ev_mid
 
@@ -320,14 +331,29 @@ def run_ours(args, w):
     hv = torch.from_numpy(vn).pin_memory()
     hout = torch.empty(qn.shape, dtype=torch.float16).pin_memory()
     e2e_steps = max(1, min(n, args.e2e_steps))
+
+    def e2e_call():
+        if qbr == 128:
+            sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+            return
+        # finer Q blocks have no host-buffer entry point: the same copies,
+        # issued from here on the same stream around the device call
+        with torch.cuda.stream(stream):
+            dq = hq.to(dev, non_blocking=True)
+            dk = hk.to(dev, non_blocking=True)
+            dv = hv.to(dev, non_blocking=True)
+            dout = torch.empty_like(dq)
+            sage.sage_attn_fwd_qblock(dq, dk, dv, dout, w.causal, sm, qbr, stream=stream)
+            hout.copy_(dout, non_blocking=True)
+
     for _ in range(2):
-        sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+        e2e_call()
     torch.cuda.synchronize(dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(e2e_steps)]
     for a, b in e2e_ev:
         a.record(stream)
-        sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+        e2e_call()
         b.record(stream)
     torch.cuda.synchronize(dev)
     sage.sage_check_device_status(stream)
@@ -349,16 +375,17 @@ def run_ours(args, w):
         achieved = ops / (attn_avg_ms * 1e-3) / 1e12
         traffic = None
         if NCU_TRAFFIC.get("attn_sha") == attn_source_hash() and \
-                NCU_TRAFFIC.get("workload") == w.name:
+                NCU_TRAFFIC.get("workload") == w.name and qbr == 128:
             traffic = NCU_TRAFFIC.get("bytes_per_launch")
-        quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d
+        quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d + 4 * B * H * -(-Lq // qbr)
         result = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "int8 QK^T (int32 acc) + fp16 PV (fp32 acc)",
             "data": "synthetic (seeded numpy N(0,1)/t4 fp16, per-channel K offsets)",
-            "config": dict(w.describe(), l2="flushed before every timed step (256 MiB write)",
+            "config": dict(w.describe(), q_block_rows=qbr,
+                           l2="flushed before every timed step (256 MiB write)",
                            parallelism=f"replicas x{world} (shard by batch/head)"),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
                          "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
@@ -379,7 +406,7 @@ def run_ours(args, w):
         torch.distributed.destroy_process_group()
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, info = time_oracle_sample(w, qn, kn, vn, args.cpu_rows, seed=0)
+        est, info = time_oracle_sample(w, qn, kn, vn, args.cpu_rows, seed=0, qbr=qbr)
         result["cpu_baseline"] = {
             "value": 4.0 * d * w.pairs() / est / 1e12, "unit": "TOPS",
             "cores": info["cores"], "kind": "oracle",
@@ -403,6 +430,8 @@ def main():
     ap.add_argument("--cpu-rows", type=int, default=2048)
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--q-block-rows", type=int, default=128, choices=[128, 64, 32, 1],
+                    help="rows per Q quantization block (finer than the 128-row tile)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     w = inputs.WORKLOADS[args.workload]

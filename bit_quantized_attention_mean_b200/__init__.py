@@ -8,6 +8,7 @@ CPU or PyTorch fallback: if the library is missing, every call raises.
 
 Exported names mirror the C ABI:
     sage_quant_qk, sage_attn_fwd, sage_attn_fwd_prequant,
+    sage_quant_qk_qblock, sage_attn_fwd_qblock, sage_attn_fwd_prequant_qblock,
     sage_quant_workspace_size, sage_attn_workspace_size,
     sage_check_device_status, sage_status_string, sage_last_launch_count
 plus two conveniences that allocate outputs: ``quant_qk`` and ``attention``.
@@ -24,12 +25,16 @@ from ._lib import (  # noqa: F401
     sage_attn_fwd_noalloc,
     NOALLOC_SCRATCH_BYTES,
     sage_attn_fwd_prequant,
+    sage_attn_fwd_prequant_qblock,
+    sage_attn_fwd_qblock,
     sage_attn_workspace_size,
     sage_check_device_status,
     sage_debug_wait_timeout,
     sage_last_launch_count,
     sage_quant_qk,
+    sage_quant_qk_qblock,
     sage_quant_workspace_size,
+    Q_BLOCK_ROWS,
     sage_status_string,
     quant_qk,
     attention,

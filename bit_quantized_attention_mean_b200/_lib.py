@@ -28,7 +28,12 @@ SYMBOLS = (
     "sage_last_launch_count",
     "sage_attn_fwd_noalloc",
     "sage_debug_wait_timeout",
+    "sage_quant_qk_qblock",
+    "sage_attn_fwd_prequant_qblock",
+    "sage_attn_fwd_qblock",
 )
+
+Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
 
 STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
           3: "SAGE_ERR_CUDA", 4: "SAGE_ERR_TIMEOUT"}
@@ -76,6 +81,14 @@ def load_library():
         lib.sage_attn_fwd_noalloc.restype = I
         lib.sage_debug_wait_timeout.argtypes = [I, P]
         lib.sage_debug_wait_timeout.restype = I
+        lib.sage_quant_qk_qblock.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, Z,
+                                             P]
+        lib.sage_quant_qk_qblock.restype = I
+        lib.sage_attn_fwd_prequant_qblock.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I,
+                                                      P]
+        lib.sage_attn_fwd_prequant_qblock.restype = I
+        lib.sage_attn_fwd_qblock.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+        lib.sage_attn_fwd_qblock.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -135,40 +148,79 @@ def sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
     return load_library().sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d)
 
 
-def sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
-                  workspace=None, stream=None):
-    """Smooth K and quantize Q/K per block into the given output tensors."""
+def _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, q_block_rows):
     import torch
-    lib = load_library()
     B, H, Hkv, Lq, Lk, d = _dims(q, k)
-    nqb, nkb = -(-Lq // 128), -(-Lk // 64)
-    args = [
+    nqb, nkb = -(-Lq // q_block_rows), -(-Lk // 64)
+    return [
         _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
         _dev(q_i8, torch.int8, "q_i8", q.shape), _dev(k_i8, torch.int8, "k_i8", k.shape),
         _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
         _dev(k_scale, torch.float32, "k_scale", (B, Hkv, nkb)),
         _dev(k_mean, torch.float32, "k_mean", (B, Hkv, d)),
+        B, H, Hkv, Lq, Lk, d,
     ]
-    if workspace is None:
-        ws, wsb = ctypes.c_void_p(0), 0
-    else:
-        ws, wsb = _dev(workspace, torch.uint8, "workspace"), workspace.numel()
-    _check(lib.sage_quant_qk(*args, B, H, Hkv, Lq, Lk, d, float(sm_scale), ws, wsb,
-                             _stream(stream)), "sage_quant_qk")
 
 
-def sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, causal, stream=None):
-    """Attention kernel on pre-quantized Q/K (fp16 V, fp16 out)."""
+def _workspace(workspace):
     import torch
-    lib = load_library()
+    if workspace is None:
+        return ctypes.c_void_p(0), 0
+    return _dev(workspace, torch.uint8, "workspace"), workspace.numel()
+
+
+def _check_qbr(q_block_rows):
+    if q_block_rows not in Q_BLOCK_ROWS:
+        raise ValueError(f"q_block_rows must be one of {Q_BLOCK_ROWS}, got {q_block_rows}")
+
+
+def sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
+                  workspace=None, stream=None):
+    """Smooth K and quantize Q/K per block into the given output tensors."""
+    args = _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, 128)
+    _check(load_library().sage_quant_qk(*args, float(sm_scale), *_workspace(workspace),
+                                        _stream(stream)), "sage_quant_qk")
+
+
+def sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, q_block_rows,
+                         workspace=None, stream=None):
+    """sage_quant_qk with Q blocks of q_block_rows rows (128, 64, 32 or 1);
+    q_scale has shape [B, H, ceil(Lq / q_block_rows)]."""
+    _check_qbr(q_block_rows)
+    args = _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, q_block_rows)
+    _check(load_library().sage_quant_qk_qblock(*args, float(sm_scale), int(q_block_rows),
+                                               *_workspace(workspace), _stream(stream)),
+           "sage_quant_qk_qblock")
+
+
+def _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows):
+    import torch
     B, H, Hkv, Lq, Lk, d = _dims(q_i8, k_i8)
-    nqb, nkb = -(-Lq // 128), -(-Lk // 64)
-    _check(lib.sage_attn_fwd_prequant(
+    nqb, nkb = -(-Lq // q_block_rows), -(-Lk // 64)
+    return [
         _dev(q_i8, torch.int8, "q_i8"), _dev(k_i8, torch.int8, "k_i8"),
         _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
         _dev(k_scale, torch.float32, "k_scale", (B, Hkv, nkb)),
         _dev(v, torch.float16, "v", k_i8.shape), _dev(out, torch.float16, "out", q_i8.shape),
-        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, _stream(stream)), "sage_attn_fwd_prequant")
+        B, H, Hkv, Lq, Lk, d,
+    ]
+
+
+def sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, causal, stream=None):
+    """Attention kernel on pre-quantized Q/K (fp16 V, fp16 out)."""
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, 128)
+    _check(load_library().sage_attn_fwd_prequant(*args, 1 if causal else 0, _stream(stream)),
+           "sage_attn_fwd_prequant")
+
+
+def sage_attn_fwd_prequant_qblock(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_block_rows,
+                                  stream=None):
+    """sage_attn_fwd_prequant for Q quantized in blocks of q_block_rows rows."""
+    _check_qbr(q_block_rows)
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
+    _check(load_library().sage_attn_fwd_prequant_qblock(*args, 1 if causal else 0,
+                                                        int(q_block_rows), _stream(stream)),
+           "sage_attn_fwd_prequant_qblock")
 
 
 def sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=None):
@@ -181,6 +233,19 @@ def sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=None):
         _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
         B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
         "sage_attn_fwd")
+
+
+def sage_attn_fwd_qblock(q, k, v, out, causal, sm_scale, q_block_rows, stream=None):
+    """sage_attn_fwd with Q quantized in blocks of q_block_rows rows."""
+    import torch
+    _check_qbr(q_block_rows)
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    _check(lib.sage_attn_fwd_qblock(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows),
+        _stream(stream)), "sage_attn_fwd_qblock")
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20
@@ -243,26 +308,37 @@ def sage_check_device_status(stream=None):
 
 # --------------------------------------------------------- conveniences
 
-def quant_qk(q, k, sm_scale, stream=None):
-    """Allocate outputs and run sage_quant_qk.
+def quant_qk(q, k, sm_scale, q_block_rows=128, stream=None):
+    """Allocate outputs and run sage_quant_qk (sage_quant_qk_qblock when
+    q_block_rows != 128).
     Returns (q_i8, k_i8, q_scale, k_scale, k_mean) as CUDA tensors."""
     import torch
+    _check_qbr(q_block_rows)
     B, H, Hkv, Lq, Lk, d = _dims(q, k)
     dev = q.device
     q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
     k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
-    q_scale = torch.empty((B, H, -(-Lq // 128)), dtype=torch.float32, device=dev)
+    q_scale = torch.empty((B, H, -(-Lq // q_block_rows)), dtype=torch.float32, device=dev)
     k_scale = torch.empty((B, Hkv, -(-Lk // 64)), dtype=torch.float32, device=dev)
     k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
-    sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, stream=stream)
+    if q_block_rows == 128:
+        sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, stream=stream)
+    else:
+        sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
+                             q_block_rows, stream=stream)
     return q_i8, k_i8, q_scale, k_scale, k_mean
 
 
-def attention(q, k, v, causal=False, sm_scale=None, stream=None):
-    """Allocate the output and run sage_attn_fwd; returns the fp16 output."""
+def attention(q, k, v, causal=False, sm_scale=None, q_block_rows=128, stream=None):
+    """Allocate the output and run sage_attn_fwd (sage_attn_fwd_qblock when
+    q_block_rows != 128); returns the fp16 output."""
     import torch
+    _check_qbr(q_block_rows)
     if sm_scale is None:
         sm_scale = q.shape[-1] ** -0.5
     out = torch.empty_like(q)
-    sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=stream)
+    if q_block_rows == 128:
+        sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=stream)
+    else:
+        sage_attn_fwd_qblock(q, k, v, out, causal, sm_scale, q_block_rows, stream=stream)
     return out

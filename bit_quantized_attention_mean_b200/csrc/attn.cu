@@ -100,7 +100,7 @@ __global__ void __launch_bounds__(192, 2)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                      const float* __restrict__ k_scale, __half* __restrict__ out, int H, int Hkv,
-                     int Lq, int Lk, int nqt, int global_lpt) {
+                     int Lq, int Lk, int nqt, int global_lpt, int qbr) {
   using C = AttnCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment of the shared-window address (swizzle atoms)
@@ -252,8 +252,9 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const int row = tid;  // warp w reads tensor-memory lanes [32w, 32w+32)
     const int qrow = q0 + row;
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const int nqb = nqt;
-    const float sq = __ldg(q_scale + (size_t)bh * nqb + qt);
+    // this row's Q scale (blocks of qbr rows; padding rows reuse the last)
+    const int nqs = (Lq + qbr - 1) / qbr;
+    const float sq = __ldg(q_scale + (size_t)bh * nqs + min(qrow, Lq - 1) / qbr);
     const float* ks = k_scale + (size_t)bhk * nkb;
     const int diag = qrow + (Lk - Lq) + 1;  // keys [0, diag) visible to this row
     float m_run = -INFINITY, l_run = 0.f;
@@ -427,7 +428,8 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launch
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.out, a.H,
                                                    a.Hkv, a.Lq, a.Lk, nqt,
-                                                   kv_bytes <= kGlobalOrderKVBytes ? 1 : 0);
+                                                   kv_bytes <= kGlobalOrderKVBytes ? 1 : 0,
+                                                   a.q_block_rows);
   *launches += 1;
   return cudaGetLastError();
 }

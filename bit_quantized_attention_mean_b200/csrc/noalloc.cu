@@ -112,12 +112,14 @@ extern "C" SAGE_API sage_status sage_attn_fwd_noalloc(const void* q, const void*
   float* k_mean = reinterpret_cast<float*>(ws + off_m);
   const float c = (float)((double)sm_scale * 1.4426950408889634074);  // sm_scale * log2(e)
   sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
-                     q_scale, k_scale, k_mean, ws + off_p, B, H, Hkv, Lq, Lk, d, c};
+                     q_scale, k_scale, k_mean, ws + off_p, B, H, Hkv, Lq, Lk, d, c,
+                     SAGE_Q_BLOCK_ROWS};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
   if (e == cudaSuccess) {
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
-                      static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1};
+                      static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,
+                      SAGE_Q_BLOCK_ROWS};
     e = sage::launch_attn(aa, s, &launches);
   }
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;

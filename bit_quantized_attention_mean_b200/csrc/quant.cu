@@ -38,24 +38,6 @@ constexpr int kCluster = 8;  // CTAs per K head (16 when there are few heads)
 
 // ------------------------------------------------------------- helpers
 
-__device__ __forceinline__ float block_absmax(float v, float* red) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float w = lane < kQuantThreads / 32 ? red[lane] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) w = fmaxf(w, __shfl_xor_sync(0xffffffffu, w, o));
-    if (lane == 0) red[8] = w;
-  }
-  __syncthreads();
-  const float a = red[8];
-  __syncthreads();  // red[] may be reused by the next block
-  return a;
-}
-
 // Abs-max of NB independent blocks at once (one value per block per thread).
 template <int NB>
 __device__ __forceinline__ void block_absmax_n(float (&v)[NB], float* red) {
@@ -109,41 +91,60 @@ __device__ __forceinline__ void values8(const uint4& raw, const float (&m)[8], f
   }
 }
 
-// Quantizes one block of `rows` x D fp16 values (row-major) into int8 and
-// returns its scale fl32(amax/127).  For K, `m` holds this thread's 8
-// channel means (the same channels for every vector of the thread).
-template <int D, int ROWS_MAX, bool SMOOTH>
-__device__ __forceinline__ float quant_block(const __half* __restrict__ src, int8_t* __restrict__ dst,
-                                             int rows, const float (&m)[8], float* red) {
-  constexpr int TPR = D / 8;                           // 16-byte vectors per row
-  constexpr int VPT = ROWS_MAX * TPR / kQuantThreads;  // vectors per thread
-  static_assert(VPT >= 1 && kQuantThreads % TPR == 0, "bad block shape");
-  const int nvec = rows * TPR;
+// Quantizes one 128-row Q tile whose quantization blocks are QBR rows
+// (QBR = 128, 64, 32 or 1) and writes ceil(rows / QBR) scales, each
+// multiplied by c.  Thread t holds, for pass v, row t / TPR + RPP * v (RPP =
+// rows per pass), so a block of QBR >= RPP rows is a group of passes reduced
+// across the CTA, and a one-row block is a group of TPR adjacent lanes.
+template <int D, int QBR>
+__device__ __forceinline__ void quant_q_tile(const __half* __restrict__ src, int8_t* __restrict__ dst,
+                                             float* __restrict__ qs, int rows, float c, float* red) {
+  constexpr int TPR = D / 8;
+  constexpr int RPP = kQuantThreads / TPR;
+  constexpr int VPT = SAGE_Q_BLOCK_ROWS / RPP;
+  static_assert(QBR == 1 || (QBR % RPP == 0 && SAGE_Q_BLOCK_ROWS % QBR == 0), "block rows");
+  constexpr int NG = QBR == 1 ? VPT : SAGE_Q_BLOCK_ROWS / QBR;  // scale groups per thread
   const int tid = threadIdx.x;
+  const int nvec = rows * TPR;
   uint4 raw[VPT];
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
     const int idx = tid + v * kQuantThreads;
     raw[v] = idx < nvec ? __ldcs(reinterpret_cast<const uint4*>(src) + idx) : make_uint4(0, 0, 0, 0);
   }
-  float amax = 0.f;
+  const float no_mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float amax[NG];
+#pragma unroll
+  for (int g = 0; g < NG; ++g) amax[g] = 0.f;
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
-    if (tid + v * kQuantThreads < nvec) {  // padding rows are not in the block
+    if (tid + v * kQuantThreads < nvec) {
       float x[8];
-      values8<SMOOTH>(raw[v], m, x);
+      values8<false>(raw[v], no_mean, x);
+      const int g = QBR == 1 ? v : v / (QBR / RPP);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(x[e]));
+      for (int e = 0; e < 8; ++e) amax[g] = fmaxf(amax[g], fabsf(x[e]));
     }
   }
-  const float a = block_absmax(amax, red);
-  const float r = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+  if (QBR == 1) {
+    // the TPR lanes of one row are adjacent within a warp
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+      for (int o = TPR / 2; o > 0; o >>= 1)
+        amax[g] = fmaxf(amax[g], __shfl_xor_sync(0xffffffffu, amax[g], o));
+  } else {
+    block_absmax_n<NG>(amax, red);
+  }
 #pragma unroll
   for (int v = 0; v < VPT; ++v) {
     const int idx = tid + v * kQuantThreads;
+    const int g = QBR == 1 ? v : v / (QBR / RPP);
+    const float a = amax[g];
+    const float r = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
     if (idx < nvec) {
       float x[8];
-      values8<SMOOTH>(raw[v], m, x);
+      values8<false>(raw[v], no_mean, x);
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
@@ -151,8 +152,12 @@ __device__ __forceinline__ float quant_block(const __half* __restrict__ src, int
       for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
       __stcs(reinterpret_cast<uint2*>(dst) + idx, make_uint2(lo, hi));
     }
+    // one thread per block writes its scale
+    const int row = idx / TPR;
+    const bool writer = QBR == 1 ? (tid % TPR == 0) : (tid == 0 && v % (QBR / RPP) == 0);
+    if (writer && row < rows)
+      qs[QBR == 1 ? row : row / QBR] = __fmul_rn(a > 0.f ? __fdiv_rn(a, 127.f) : 0.f, c);
   }
-  return a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
 }
 
 // Smooths and quantizes NB consecutive K blocks [kb, kb+NB) of one head
@@ -217,7 +222,7 @@ __device__ __forceinline__ void quant_k_blocks(const __half* __restrict__ kh, in
 
 // ------------------------------------------------------------- kernel
 
-template <int D>
+template <int D, int QBR>
 __global__ void __launch_bounds__(kQuantThreads)
 quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
                 int8_t* __restrict__ q_i8, int8_t* __restrict__ k_i8,
@@ -231,7 +236,6 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   __shared__ long long rsum[RPP * D > 0 ? RPP * D : 1];
   __shared__ float mean[D];
   const int tid = threadIdx.x;
-  const float no_mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 
   if ((int)blockIdx.x >= n_k_ctas) {
     // ------------------------------------------------------------ Q block
@@ -240,9 +244,9 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
     const int bh = blk / nqb, qb = blk - bh * nqb;
     const int r0 = qb * SAGE_Q_BLOCK_ROWS;
     const size_t off = ((size_t)bh * Lq + r0) * D;
-    const float s = quant_block<D, SAGE_Q_BLOCK_ROWS, false>(
-        q + off, q_i8 + off, min(SAGE_Q_BLOCK_ROWS, Lq - r0), no_mean, red);
-    if (tid == 0) q_scale[blk] = __fmul_rn(s, c);
+    const int nqs = (Lq + QBR - 1) / QBR;  // scales per head
+    quant_q_tile<D, QBR>(q + off, q_i8 + off, q_scale + (size_t)bh * nqs + r0 / QBR,
+                         min(SAGE_Q_BLOCK_ROWS, Lq - r0), c, red);
     return;
   }
 
@@ -303,12 +307,12 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
 
 size_t quant_workspace_bytes(int, int, int, int) { return 0; }
 
-template <int D>
+template <int D, int QBR>
 static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* launches) {
   const int BH = a.B * a.H, BHkv = a.B * a.Hkv;
   const int nqb = (a.Lq + SAGE_Q_BLOCK_ROWS - 1) / SAGE_Q_BLOCK_ROWS;
   const int nkb = (a.Lk + SAGE_K_BLOCK_ROWS - 1) / SAGE_K_BLOCK_ROWS;
-  auto kern = quant_qk_kernel<D>;
+  auto kern = quant_qk_kernel<D, QBR>;
   // few heads: wider clusters so the K work spreads over more SMs
   int cl = kCluster;
   if ((long long)BHkv * kCluster < 256 &&
@@ -343,8 +347,20 @@ static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* laun
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_quant_qbr(const QuantArgs& a, cudaStream_t st, int* launches) {
+  switch (a.q_block_rows) {
+    case 128: return launch_quant_d<D, 128>(a, st, launches);
+    case 64: return launch_quant_d<D, 64>(a, st, launches);
+    case 32: return launch_quant_d<D, 32>(a, st, launches);
+    case 1: return launch_quant_d<D, 1>(a, st, launches);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_quant(const QuantArgs& a, cudaStream_t st, int* launches) {
-  return a.d == 128 ? launch_quant_d<128>(a, st, launches) : launch_quant_d<64>(a, st, launches);
+  return a.d == 128 ? launch_quant_qbr<128>(a, st, launches)
+                    : launch_quant_qbr<64>(a, st, launches);
 }
 
 }  // namespace sage

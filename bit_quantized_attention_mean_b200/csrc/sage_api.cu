@@ -47,9 +47,9 @@ struct AttnWorkspace {
   size_t q_i8, k_i8, q_scale, k_scale, k_mean, part, total;
 };
 
-AttnWorkspace attn_workspace_layout(int B, int H, int Hkv, int Lq, int Lk, int d) {
+AttnWorkspace attn_workspace_layout(int B, int H, int Hkv, int Lq, int Lk, int d, int qbr) {
   AttnWorkspace w;
-  const size_t nqb = (size_t)(Lq + 127) / 128, nkb = (size_t)(Lk + 63) / 64;
+  const size_t nqb = (size_t)(Lq + qbr - 1) / qbr, nkb = (size_t)(Lk + 63) / 64;
   size_t off = 0;
   w.q_i8 = off;    off += round_up((size_t)B * H * Lq * d);
   w.k_i8 = off;    off += round_up((size_t)B * Hkv * Lk * d);
@@ -85,16 +85,25 @@ size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d) {
 
 size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
   if (check_shape(B, H, Hkv, Lq, Lk, d) != SAGE_OK) return 0;
-  return attn_workspace_layout(B, H, Hkv, Lq, Lk, d).total;
+  return attn_workspace_layout(B, H, Hkv, Lq, Lk, d, SAGE_Q_BLOCK).total;
 }
 
 sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale,
                           float* k_scale, float* k_mean, int B, int H, int Hkv, int Lq, int Lk,
                           int d, float sm_scale, void* workspace, size_t workspace_bytes,
                           void* stream) {
+  return sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, B, H, Hkv, Lq, Lk, d,
+                              sm_scale, SAGE_Q_BLOCK, workspace, workspace_bytes, stream);
+}
+
+sage_status sage_quant_qk_qblock(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8,
+                                 float* q_scale, float* k_scale, float* k_mean, int B, int H,
+                                 int Hkv, int Lq, int Lk, int d, float sm_scale, int q_block_rows,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !q_i8 || !k_i8 || !q_scale || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8) ||
       !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(k_mean))
@@ -109,7 +118,8 @@ sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_
   const bool own = !ws && need > 0;
   if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
   sage::QuantArgs a{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
-                    q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale)};
+                    q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale),
+                    q_block_rows};
   int launches = 0;
   cudaError_t e = sage::launch_quant(a, s, &launches);
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
@@ -120,9 +130,19 @@ sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_
 sage_status sage_attn_fwd_prequant(const int8_t* q_i8, const int8_t* k_i8, const float* q_scale,
                                    const float* k_scale, const void* v, void* out, int B, int H,
                                    int Hkv, int Lq, int Lk, int d, int causal, void* stream) {
+  return sage_attn_fwd_prequant_qblock(q_i8, k_i8, q_scale, k_scale, v, out, B, H, Hkv, Lq, Lk, d,
+                                       causal, SAGE_Q_BLOCK, stream);
+}
+
+sage_status sage_attn_fwd_prequant_qblock(const int8_t* q_i8, const int8_t* k_i8,
+                                          const float* q_scale, const float* k_scale,
+                                          const void* v, void* out, int B, int H, int Hkv, int Lq,
+                                          int Lk, int d, int causal, int q_block_rows,
+                                          void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
       !aligned16(q_scale) || !aligned16(k_scale))
@@ -130,7 +150,7 @@ sage_status sage_attn_fwd_prequant(const int8_t* q_i8, const int8_t* k_i8, const
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if ((st = check_device()) != SAGE_OK) return st;
   sage::AttnArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
-                   static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1};
+                   static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows};
   int launches = 0;
   cudaError_t e = sage::launch_attn(a, static_cast<cudaStream_t>(stream), &launches);
   g_last_launches = launches;
@@ -140,9 +160,17 @@ sage_status sage_attn_fwd_prequant(const int8_t* q_i8, const int8_t* k_i8, const
 sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out, int B, int H,
                           int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
                           void* stream) {
+  return sage_attn_fwd_qblock(q, k, v, out, B, H, Hkv, Lq, Lk, d, causal, sm_scale, SAGE_Q_BLOCK,
+                              stream);
+}
+
+sage_status sage_attn_fwd_qblock(const void* q, const void* k, const void* v, void* out, int B,
+                                 int H, int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
+                                 int q_block_rows, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return SAGE_ERR_INVALID_ARG;
@@ -151,7 +179,7 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out
   if ((st = check_device()) != SAGE_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const AttnWorkspace w = attn_workspace_layout(B, H, Hkv, Lq, Lk, d);
+  const AttnWorkspace w = attn_workspace_layout(B, H, Hkv, Lq, Lk, d, q_block_rows);
   char* ws = nullptr;
   if (cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, s) != cudaSuccess)
     return SAGE_ERR_CUDA;
@@ -162,12 +190,13 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out
   float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
   sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
                      q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
-                     fold_constant(sm_scale)};
+                     fold_constant(sm_scale), q_block_rows};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
   if (e == cudaSuccess) {
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
-                      static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1};
+                      static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,
+                      q_block_rows};
     e = sage::launch_attn(aa, s, &launches);
   }
   if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;

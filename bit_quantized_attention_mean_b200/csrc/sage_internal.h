@@ -24,6 +24,7 @@ struct QuantArgs {
   void* workspace;  // quant_workspace_bytes() of scratch (int64 partial sums)
   int B, H, Hkv, Lq, Lk, d;
   float c;          // fl32(double(sm_scale) * log2(e)), folded into q_scale
+  int q_block_rows; // rows per Q quantization block: 128, 64, 32 or 1
 };
 
 struct AttnArgs {
@@ -35,7 +36,10 @@ struct AttnArgs {
   __half* out;
   int B, H, Hkv, Lq, Lk, d;
   bool causal;
+  int q_block_rows; // rows per q_scale entry: 128, 64, 32 or 1
 };
+
+inline bool valid_q_block_rows(int r) { return r == 128 || r == 64 || r == 32 || r == 1; }
 
 size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d);
 

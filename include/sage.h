@@ -90,6 +90,29 @@ SAGE_API sage_status sage_quant_qk(const void *q, const void *k,
                           float sm_scale, void *workspace, size_t workspace_bytes,
                           void *stream);
 
+/*
+ * sage_quant_qk_qblock -- sage_quant_qk with a finer Q granularity.
+ *
+ * The list of techniques in "Berkeley AI 转发研究注意力计算 8 位、4 位量化可对齐
+ * FP32 精度基线" (the key-points list) and the SageAttention2 description in
+ * the SageAttention article name quantization blocks smaller than the
+ * attention tile; here Q blocks of q_block_rows rows, one of 128 (the tile,
+ * identical to sage_quant_qk), 64, 32 or 1 (one scale per query token).
+ * Every block lies inside one 128-row attention tile, so the tiles and the
+ * kernels that consume them are unchanged; only the number of Q scales
+ * grows.  K keeps its 64-row blocks.
+ *
+ *   q_scale  fp32 [B, H, ceil(Lq/q_block_rows)]  (out) same formula per block
+ *   every other argument: as sage_quant_qk.
+ * Returns SAGE_ERR_INVALID_ARG for any other q_block_rows.
+ */
+SAGE_API sage_status sage_quant_qk_qblock(const void *q, const void *k,
+                          int8_t *q_i8, int8_t *k_i8,
+                          float *q_scale, float *k_scale, float *k_mean,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          float sm_scale, int q_block_rows,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of scratch sage_quant_qk needs (currently 0). */
 SAGE_API size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d);
 
@@ -111,6 +134,18 @@ SAGE_API sage_status sage_attn_fwd_prequant(const int8_t *q_i8, const int8_t *k_
                                    int causal, void *stream);
 
 /*
+ * sage_attn_fwd_prequant_qblock -- sage_attn_fwd_prequant for Q quantized by
+ * sage_quant_qk_qblock with the same q_block_rows (128, 64, 32 or 1): row i
+ * of head (b, h) is dequantized with q_scale[b, h, i / q_block_rows].
+ * Returns SAGE_ERR_INVALID_ARG for any other q_block_rows.
+ */
+SAGE_API sage_status sage_attn_fwd_prequant_qblock(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows, void *stream);
+
+/*
  * sage_attn_fwd -- the whole forward pass (steps 1-5) on fp16 Q, K, V.
  *   q fp16 [B, H, Lq, d], k/v fp16 [B, Hkv, Lk, d], out fp16 [B, H, Lq, d].
  * Scratch (int8 Q/K, scales, mean, partial sums;
@@ -120,6 +155,17 @@ SAGE_API sage_status sage_attn_fwd_prequant(const int8_t *q_i8, const int8_t *k_
 SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *out,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
                           int causal, float sm_scale, void *stream);
+
+/*
+ * sage_attn_fwd_qblock -- sage_attn_fwd with Q quantized in blocks of
+ * q_block_rows rows (128, 64, 32 or 1; see sage_quant_qk_qblock).  Its
+ * scratch, allocated and released on `stream` like sage_attn_fwd's, is at
+ * most sage_attn_workspace_size() + 4*B*H*Lq + 256 bytes (the Q scales grow
+ * to ceil(Lq/q_block_rows) per head).
+ */
+SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const void *v, void *out,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          int causal, float sm_scale, int q_block_rows, void *stream);
 
 /*
  * sage_attn_fwd_host -- sage_attn_fwd on HOST buffers, for callers whose data

@@ -3,6 +3,7 @@ exports exactly what include/sage.h declares (no compute calls here)."""
 import ctypes
 import os
 import re
+import pytest
 
 import bit_quantized_attention_mean_b200 as sage
 
@@ -35,3 +36,13 @@ def test_host_only_helpers():
     assert sage.sage_attn_workspace_size(1, 3, 2, 256, 256, 64) == 0   # H % Hkv != 0
     # the K mean is reduced on chip: no scratch
     assert sage.sage_quant_workspace_size(2, 4, 1000, 128) == 0
+
+
+def test_binding_rejects_unsupported_q_block_rows_before_any_call():
+    import bit_quantized_attention_mean_b200 as sage
+    assert sage.Q_BLOCK_ROWS == (128, 64, 32, 1)
+    for bad in (0, 16, 100, 256):
+        with pytest.raises(ValueError):
+            sage.attention(None, None, None, q_block_rows=bad)
+        with pytest.raises(ValueError):
+            sage.quant_qk(None, None, 0.1, q_block_rows=bad)
