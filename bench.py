@@ -52,8 +52,8 @@ INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "4db0ac417f080078", "workload": "llm-causal-B1H32L4096d128",
-               "bytes_per_launch": 68573184 + 7489792}
+NCU_TRAFFIC = {"attn_sha": "792aafd858761851", "workload": "llm-causal-B1H32L4096d128",
+               "bytes_per_launch": 68349184 + 6456576}
 
 
 def load_peaks():
