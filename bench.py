@@ -1,7 +1,7 @@
 """Benchmark of the 8-bit quantized attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 1..5] [--q-block-rows 128|64|32|1]
+                    [--workload 1..5] [--q-block-rows 128|64|32|1] [--pv-accum f32|f16]
 
 A step is one pass of the whole hot path over the workload: K mean + Q/K
 quantization (sage_quant_qk) and the fused attention kernel
@@ -15,7 +15,9 @@ PV work counted at 2*d each.  ``e2e`` is the same metric through the public
 host-buffer call (sage_attn_fwd_host: H2D of q/k/v, forward pass, D2H of the
 output, all inside the timed region).  ``--q-block-rows`` quantizes Q in
 blocks finer than the 128-row attention tile (the _qblock entry points; e2e
-then issues the same copies around sage_attn_fwd_qblock).  ``roofline`` reports the attention
+then issues the same copies around sage_attn_fwd_ex); ``--pv-accum f16``
+sums P V in fp16 as the SageAttention article states (sage_attn_fwd_ex /
+sage_attn_fwd_prequant_ex with SAGE_PV_ACCUM_F16).  ``roofline`` reports the attention
 kernel against the combined tensor roofline: QK at the INT8 peak and PV at the
 FP16 peak, t_roof = 2*d*pairs/P_int8 + 2*d*pairs/P_fp16, with P_fp16 the
 measured bf16 peak and P_int8 = 2 x P_fp16 (nominal dense ratio).
@@ -229,7 +231,8 @@ def run_reference(args, w):
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (int8 codes, int32 dot products)",
         "data": "synthetic (seeded numpy, fp16)",
-        "config": dict(w.describe(), q_block_rows=args.q_block_rows, l2="n/a (CPU)"),
+        "config": dict(w.describe(), q_block_rows=args.q_block_rows, pv_accum=args.pv_accum,
+                       l2="n/a (CPU)"),
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": info["cores"],
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
@@ -287,7 +290,10 @@ def run_ours(args, w):
         launches += sage.sage_last_launch_count()
         ev_mid = torch.cuda.Event(enable_timing=True)
         ev_mid.record(stream)
-        if qbr == 128:
+        if args.pv_accum != "f32":
+            sage.sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, w.causal, qbr,
+                                           args.pv_accum, stream=stream)
+        elif qbr == 128:
             sage.sage_attn_fwd_prequant(q_i8, k_i8, q_scale, k_scale, v, out, w.causal,
                                         stream=stream)
         else:
@@ -333,7 +339,7 @@ def run_ours(args, w):
     e2e_steps = max(1, min(n, args.e2e_steps))
 
     def e2e_call():
-        if qbr == 128:
+        if qbr == 128 and args.pv_accum == "f32":
             sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
             return
         # finer Q blocks have no host-buffer entry point: the same copies,
@@ -343,7 +349,8 @@ def run_ours(args, w):
             dk = hk.to(dev, non_blocking=True)
             dv = hv.to(dev, non_blocking=True)
             dout = torch.empty_like(dq)
-            sage.sage_attn_fwd_qblock(dq, dk, dv, dout, w.causal, sm, qbr, stream=stream)
+            sage.sage_attn_fwd_ex(dq, dk, dv, dout, w.causal, sm, qbr, args.pv_accum,
+                                  stream=stream)
             hout.copy_(dout, non_blocking=True)
 
     for _ in range(2):
@@ -375,16 +382,17 @@ def run_ours(args, w):
         achieved = ops / (attn_avg_ms * 1e-3) / 1e12
         traffic = None
         if NCU_TRAFFIC.get("attn_sha") == attn_source_hash() and \
-                NCU_TRAFFIC.get("workload") == w.name and qbr == 128:
+                NCU_TRAFFIC.get("workload") == w.name and qbr == 128 and \
+                args.pv_accum == "f32":
             traffic = NCU_TRAFFIC.get("bytes_per_launch")
         quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d + 4 * B * H * -(-Lq // qbr)
         result = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "int8 QK^T (int32 acc) + fp16 PV (fp32 acc)",
+            "dtype": f"int8 QK^T (int32 acc) + fp16 PV ({args.pv_accum} acc)",
             "data": "synthetic (seeded numpy N(0,1)/t4 fp16, per-channel K offsets)",
-            "config": dict(w.describe(), q_block_rows=qbr,
+            "config": dict(w.describe(), q_block_rows=qbr, pv_accum=args.pv_accum,
                            l2="flushed before every timed step (256 MiB write)",
                            parallelism=f"replicas x{world} (shard by batch/head)"),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
@@ -432,6 +440,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-block-rows", type=int, default=128, choices=[128, 64, 32, 1],
                     help="rows per Q quantization block (finer than the 128-row tile)")
+    ap.add_argument("--pv-accum", default="f32", choices=["f32", "f16"],
+                    help="P V accumulator: fp32 (default) or fp16 as the article states")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
     w = inputs.WORKLOADS[args.workload]

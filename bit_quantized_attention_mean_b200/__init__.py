@@ -9,6 +9,7 @@ CPU or PyTorch fallback: if the library is missing, every call raises.
 Exported names mirror the C ABI:
     sage_quant_qk, sage_attn_fwd, sage_attn_fwd_prequant,
     sage_quant_qk_qblock, sage_attn_fwd_qblock, sage_attn_fwd_prequant_qblock,
+    sage_attn_fwd_ex, sage_attn_fwd_prequant_ex,
     sage_quant_workspace_size, sage_attn_workspace_size,
     sage_check_device_status, sage_status_string, sage_last_launch_count
 plus two conveniences that allocate outputs: ``quant_qk`` and ``attention``.
@@ -27,6 +28,10 @@ from ._lib import (  # noqa: F401
     sage_attn_fwd_prequant,
     sage_attn_fwd_prequant_qblock,
     sage_attn_fwd_qblock,
+    sage_attn_fwd_ex,
+    sage_attn_fwd_prequant_ex,
+    SAGE_PV_ACCUM_F16,
+    PV_ACCUM,
     sage_attn_workspace_size,
     sage_check_device_status,
     sage_debug_wait_timeout,

@@ -31,9 +31,13 @@ SYMBOLS = (
     "sage_quant_qk_qblock",
     "sage_attn_fwd_prequant_qblock",
     "sage_attn_fwd_qblock",
+    "sage_attn_fwd_ex",
+    "sage_attn_fwd_prequant_ex",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
+SAGE_PV_ACCUM_F16 = 1             # flag of the _ex calls: fp16 P V accumulator
+PV_ACCUM = {"f32": 0, "f16": SAGE_PV_ACCUM_F16}
 
 STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
           3: "SAGE_ERR_CUDA", 4: "SAGE_ERR_TIMEOUT"}
@@ -89,6 +93,11 @@ def load_library():
         lib.sage_attn_fwd_prequant_qblock.restype = I
         lib.sage_attn_fwd_qblock.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, P]
         lib.sage_attn_fwd_qblock.restype = I
+        U = ctypes.c_uint
+        lib.sage_attn_fwd_ex.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, U, P]
+        lib.sage_attn_fwd_ex.restype = I
+        lib.sage_attn_fwd_prequant_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, P]
+        lib.sage_attn_fwd_prequant_ex.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -248,6 +257,39 @@ def sage_attn_fwd_qblock(q, k, v, out, causal, sm_scale, q_block_rows, stream=No
         _stream(stream)), "sage_attn_fwd_qblock")
 
 
+def _flags(pv_accum):
+    if pv_accum not in PV_ACCUM:
+        raise ValueError(f"pv_accum must be one of {tuple(PV_ACCUM)}, got {pv_accum!r}")
+    return PV_ACCUM[pv_accum]
+
+
+def sage_attn_fwd_ex(q, k, v, out, causal, sm_scale, q_block_rows=128, pv_accum="f32",
+                     stream=None):
+    """sage_attn_fwd with a Q block height and the P V accumulator ("f32",
+    the default, or "f16" as the SageAttention article states)."""
+    import torch
+    _check_qbr(q_block_rows)
+    flags = _flags(pv_accum)
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    _check(lib.sage_attn_fwd_ex(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows), flags,
+        _stream(stream)), "sage_attn_fwd_ex")
+
+
+def sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_block_rows=128,
+                              pv_accum="f32", stream=None):
+    """sage_attn_fwd_prequant_qblock with the P V accumulator selectable."""
+    _check_qbr(q_block_rows)
+    flags = _flags(pv_accum)
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
+    _check(load_library().sage_attn_fwd_prequant_ex(*args, 1 if causal else 0,
+                                                    int(q_block_rows), flags, _stream(stream)),
+           "sage_attn_fwd_prequant_ex")
+
+
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
@@ -329,15 +371,20 @@ def quant_qk(q, k, sm_scale, q_block_rows=128, stream=None):
     return q_i8, k_i8, q_scale, k_scale, k_mean
 
 
-def attention(q, k, v, causal=False, sm_scale=None, q_block_rows=128, stream=None):
+def attention(q, k, v, causal=False, sm_scale=None, q_block_rows=128, pv_accum="f32",
+              stream=None):
     """Allocate the output and run sage_attn_fwd (sage_attn_fwd_qblock when
-    q_block_rows != 128); returns the fp16 output."""
+    q_block_rows != 128, sage_attn_fwd_ex for an fp16 P V accumulator);
+    returns the fp16 output."""
     import torch
     _check_qbr(q_block_rows)
+    _flags(pv_accum)
     if sm_scale is None:
         sm_scale = q.shape[-1] ** -0.5
     out = torch.empty_like(q)
-    if q_block_rows == 128:
+    if pv_accum != "f32":
+        sage_attn_fwd_ex(q, k, v, out, causal, sm_scale, q_block_rows, pv_accum, stream=stream)
+    elif q_block_rows == 128:
         sage_attn_fwd(q, k, v, out, causal, sm_scale, stream=stream)
     else:
         sage_attn_fwd_qblock(q, k, v, out, causal, sm_scale, q_block_rows, stream=stream)

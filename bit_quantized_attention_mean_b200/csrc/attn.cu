@@ -28,6 +28,12 @@
 // MMAs.  tcgen05 operations from one thread execute in issue order, which is
 // what makes reusing a score buffer for S_{j+2} after P_j V_j safe.
 //
+// F16ACC selects the accumulator the article names for P V ("对 P, V 采用
+// FP16 数据类型的矩阵乘法累加器"): the P V products accumulate in fp16 (one value
+// per tensor-memory column, in its low half), and the running max is exact
+// (O rescaled whenever it grows) so that P <= 1 keeps the sums in fp16 range.
+// The default accumulates in fp32.
+//
 // Tensor memory (256 columns): [0,64) S/P buffer 0, [64,128) S/P buffer 1,
 // [128,128+d) O accumulator.  Every mbarrier wait is bounded (2 s); on expiry
 // the CTA stops issuing work, drains what is in flight, frees its tensor
@@ -88,6 +94,18 @@ struct AttnCfg {
                 "tiles must stay 1024-byte aligned");
 };
 
+// An accumulator column as fp32: fp32 sums hold the value itself, fp16 sums
+// an fp16 value in the low half.
+template <bool F16ACC>
+__device__ __forceinline__ float acc_value(uint32_t col) {
+  return F16ACC ? __half2float(__ushort_as_half((unsigned short)(col & 0xffffu))) : __uint_as_float(col);
+}
+
+// An fp16 accumulator column multiplied by alpha (rounded back to fp16).
+__device__ __forceinline__ uint32_t acc16_scale(uint32_t col, float alpha) {
+  return (uint32_t)__half_as_ushort(__float2half_rn(acc_value<true>(col) * alpha));
+}
+
 // Warp-uniform bounded wait: every lane waits, then the warp agrees.
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           int site, uint64_t limit_ns = kWaitLimitNs) {
@@ -95,7 +113,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16ACC>
 __global__ void __launch_bounds__(192, 2)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
@@ -190,7 +208,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && nkt > 0) {
       constexpr uint32_t idesc_qk = make_idesc_i8(BQ, BK);
-      constexpr uint32_t idesc_pv = make_idesc_f16(BQ, D, /*b_mn_major=*/true);
+      constexpr uint32_t idesc_pv = make_idesc_f16(BQ, D, /*b_mn_major=*/true, F16ACC);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q);
       auto issue_pv = [&](int jj) -> bool {
         const int bb = jj & 1, ss = jj % C::STAGES;
@@ -286,7 +304,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       }
       // |S| <= 127*127*128 < 2^22, so the int -> float conversion is exact
       const float mt = vis > 0 ? (float)mx * c : -INFINITY;
-      const bool need = mt > m_run + 8.0f;
+      // rescale threshold (base 2): lazy for fp32 sums, exact for fp16 sums
+      const bool need = mt > m_run + (F16ACC ? 0.0f : 8.0f);
       float alpha = 1.f;
       if (need) {
         alpha = ex2_approx(m_run - mt);  // 0 when m_run = -inf
@@ -305,7 +324,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + C::O_COL + cc * 32, o);
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          for (int i = 0; i < 32; ++i) o[i] = F16ACC ? acc16_scale(o[i], alpha)
+                                                      : __float_as_uint(__uint_as_float(o[i]) * alpha);
           tmem_st32(tmem + lane_base + C::O_COL + cc * 32, o);
         }
       }
@@ -353,7 +373,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         uint32_t hv[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
-          hv[i] = pack_half2(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+          hv[i] = pack_half2(acc_value<F16ACC>(o[2 * i]) * inv, acc_value<F16ACC>(o[2 * i + 1]) * inv);
         if (qrow < Lq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
@@ -402,10 +422,10 @@ static bool make_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool F16ACC>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launches) {
   using C = AttnCfg<D>;
-  auto kern = sage_attn_fwd_kernel<D, CAUSAL>;
+  auto kern = sage_attn_fwd_kernel<D, CAUSAL, F16ACC>;
   // per device context; cheap enough to repeat on every launch
   cudaError_t attr_err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -434,12 +454,18 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launch
   return cudaGetLastError();
 }
 
-cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches) {
+template <bool F16ACC>
+static cudaError_t launch_attn_acc(const AttnArgs& a, cudaStream_t st, int* launches) {
   if (a.d == 128)
-    return a.causal ? launch_attn_t<128, true>(a, st, launches)
-                    : launch_attn_t<128, false>(a, st, launches);
-  return a.causal ? launch_attn_t<64, true>(a, st, launches)
-                  : launch_attn_t<64, false>(a, st, launches);
+    return a.causal ? launch_attn_t<128, true, F16ACC>(a, st, launches)
+                    : launch_attn_t<128, false, F16ACC>(a, st, launches);
+  return a.causal ? launch_attn_t<64, true, F16ACC>(a, st, launches)
+                  : launch_attn_t<64, false, F16ACC>(a, st, launches);
+}
+
+cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches) {
+  return a.pv_f16_accum ? launch_attn_acc<true>(a, st, launches)
+                        : launch_attn_acc<false>(a, st, launches);
 }
 
 // One warp waits on an mbarrier that nothing ever completes, through the

@@ -139,10 +139,19 @@ sage_status sage_attn_fwd_prequant_qblock(const int8_t* q_i8, const int8_t* k_i8
                                           const void* v, void* out, int B, int H, int Hkv, int Lq,
                                           int Lk, int d, int causal, int q_block_rows,
                                           void* stream) {
+  return sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, B, H, Hkv, Lq, Lk, d,
+                                   causal, q_block_rows, 0u, stream);
+}
+
+sage_status sage_attn_fwd_prequant_ex(const int8_t* q_i8, const int8_t* k_i8,
+                                      const float* q_scale, const float* k_scale, const void* v,
+                                      void* out, int B, int H, int Hkv, int Lq, int Lk, int d,
+                                      int causal, int q_block_rows, unsigned flags, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if ((flags & ~(unsigned)SAGE_PV_ACCUM_F16) != 0u) return SAGE_ERR_INVALID_ARG;
   if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
       !aligned16(q_scale) || !aligned16(k_scale))
@@ -150,7 +159,8 @@ sage_status sage_attn_fwd_prequant_qblock(const int8_t* q_i8, const int8_t* k_i8
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if ((st = check_device()) != SAGE_OK) return st;
   sage::AttnArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
-                   static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows};
+                   static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows,
+                   (flags & SAGE_PV_ACCUM_F16) != 0u};
   int launches = 0;
   cudaError_t e = sage::launch_attn(a, static_cast<cudaStream_t>(stream), &launches);
   g_last_launches = launches;
@@ -167,10 +177,18 @@ sage_status sage_attn_fwd(const void* q, const void* k, const void* v, void* out
 sage_status sage_attn_fwd_qblock(const void* q, const void* k, const void* v, void* out, int B,
                                  int H, int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
                                  int q_block_rows, void* stream) {
+  return sage_attn_fwd_ex(q, k, v, out, B, H, Hkv, Lq, Lk, d, causal, sm_scale, q_block_rows, 0u,
+                          stream);
+}
+
+sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int H,
+                             int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
+                             int q_block_rows, unsigned flags, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if ((flags & ~(unsigned)SAGE_PV_ACCUM_F16) != 0u) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return SAGE_ERR_INVALID_ARG;
@@ -196,7 +214,7 @@ sage_status sage_attn_fwd_qblock(const void* q, const void* k, const void* v, vo
   if (e == cudaSuccess) {
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                       static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,
-                      q_block_rows};
+                      q_block_rows, (flags & SAGE_PV_ACCUM_F16) != 0u};
     e = sage::launch_attn(aa, s, &launches);
   }
   if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;

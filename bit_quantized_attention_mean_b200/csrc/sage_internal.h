@@ -36,7 +36,8 @@ struct AttnArgs {
   __half* out;
   int B, H, Hkv, Lq, Lk, d;
   bool causal;
-  int q_block_rows; // rows per q_scale entry: 128, 64, 32 or 1
+  int q_block_rows;   // rows per q_scale entry: 128, 64, 32 or 1
+  bool pv_f16_accum;  // accumulate P V in fp16 (else fp32)
 };
 
 inline bool valid_q_block_rows(int r) { return r == 128 || r == 64 || r == 32 || r == 1; }

@@ -182,10 +182,12 @@ __host__ __device__ constexpr uint32_t make_idesc_i8(int M, int N) {
          ((uint32_t)(M >> 4) << 24);
 }
 
-// kind::f16, F16 x F16 -> F32; A K-major (A may come from tensor memory),
-// B major given by b_mn_major.
-__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, bool b_mn_major) {
-  return (1u << 4) | (0u << 7) | (0u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
+// kind::f16, F16 x F16 -> F32 (or F16 when d_f16); A K-major (A may come from
+// tensor memory), B major given by b_mn_major.  An F16 D keeps one value per
+// tensor-memory column, in the low 16 bits.
+__host__ __device__ constexpr uint32_t make_idesc_f16(int M, int N, bool b_mn_major,
+                                                      bool d_f16 = false) {
+  return ((d_f16 ? 0u : 1u) << 4) | (0u << 7) | (0u << 10) | ((b_mn_major ? 1u : 0u) << 16) |
          ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
 

@@ -61,6 +61,9 @@ typedef enum {
 #define SAGE_Q_BLOCK 128
 #define SAGE_K_BLOCK 64
 
+/* Flags of the _ex entry points. */
+#define SAGE_PV_ACCUM_F16 1u  /* accumulate P V in fp16 (the article's choice) */
+
 /*
  * sage_quant_qk -- steps 1-2: smoothing of K and per-block INT8 quantization.
  *
@@ -166,6 +169,28 @@ SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, 
 SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const void *v, void *out,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
                           int causal, float sm_scale, int q_block_rows, void *stream);
+
+/*
+ * sage_attn_fwd_ex / sage_attn_fwd_prequant_ex -- the _qblock entry points
+ * with a flags word.  SAGE_PV_ACCUM_F16 selects the P V accumulator the
+ * SageAttention article states ("对 P, V 采用 FP16 数据类型的矩阵乘法累加器",
+ * method section): P and V stay fp16 and their products are summed in fp16
+ * (the tensor core's F16 D format) instead of fp32.  With it the running
+ * row max is kept exact (O is rescaled whenever it grows), so P <= 1 and, as
+ * the article argues, the sums stay within the fp16 range; the result is
+ * less accurate than the fp32 default (the error grows with Lk) and no
+ * faster on this GPU.  flags = 0 is identical to the _qblock calls.  Any
+ * other bit returns SAGE_ERR_INVALID_ARG.
+ */
+SAGE_API sage_status sage_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          int causal, float sm_scale, int q_block_rows, unsigned flags,
+                          void *stream);
+SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows, unsigned flags, void *stream);
 
 /*
  * sage_attn_fwd_host -- sage_attn_fwd on HOST buffers, for callers whose data
