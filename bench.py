@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                     [--workload 1..5] [--q-block-rows 128|64|32|1] [--pv-accum f32|f16]
+                    [--decode]
 
 A step is one pass of the whole hot path over the workload: K mean + Q/K
 quantization (sage_quant_qk) and the fused attention kernel
@@ -427,6 +428,87 @@ def run_ours(args, w):
     return 0
 
 
+DECODE_SHAPE = {"B": 8, "H": 32, "Hkv": 8, "Lq": 1, "Lk": 32768, "d": 128}
+
+
+def run_decode_bench(args):
+    """Decoding step: one query token per head against a 32768-token KV cache
+    that is already quantized (int8 K, fp16 V resident in HBM); times
+    sage_attn_decode_prequant (decode kernel + split merge) against the HBM
+    roofline.  Single GPU, rank 0 prints."""
+    import torch
+    import bit_quantized_attention_mean_b200 as sage
+
+    world, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    sh = DECODE_SHAPE
+    B, H, Hkv, Lq, Lk, d = sh["B"], sh["H"], sh["Hkv"], sh["Lq"], sh["Lk"], sh["d"]
+    qn, kn, vn = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=93, k_offset_sigma=1.0)
+    sm = float(np.float32(1 / np.sqrt(d)))
+    q, k, v = (torch.from_numpy(x).to(dev) for x in (qn, kn, vn))
+    qi, ki, qs, ks, km = sage.quant_qk(q, k, sm, q_block_rows=1)   # the cache, quantized once
+    del k
+    out = torch.empty_like(q)
+    ws = torch.empty(max(16, sage.sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d)),
+                     dtype=torch.uint8, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    launches = 0
+
+    def step():
+        nonlocal launches
+        sage.sage_attn_decode_prequant(qi, ki, qs, ks, v, out, True, 1, workspace=ws,
+                                       stream=stream)
+        launches += sage.sage_last_launch_count()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    sage.sage_check_device_status(stream)
+    n = args.steps
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    torch.cuda.synchronize(dev)
+    launches = 0
+    with ClockSampler(local) as clocks:
+        for i in range(n):
+            flush.zero_()
+            evs[i][0].record(stream)
+            step()
+            evs[i][1].record(stream)
+        torch.cuda.synchronize(dev)
+    sage.sage_check_device_status(stream)
+    ms = float(sum(a.elapsed_time(b) for a, b in evs) / n)
+    if rank != 0:
+        return 0
+    pairs = inputs.visible_pairs(B, H, Lq, Lk, True)
+    ops = 4.0 * d * pairs
+    nbytes = (ki.numel() + 2 * v.numel() + qi.numel() + 2 * out.numel()
+              + 4 * (qs.numel() + ks.numel()))
+    peaks = load_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": "quantized attention decode TOPS at 1 B200 and % of HBM roofline",
+        "value": ops / (ms * 1e-3) / 1e12, "unit": "TOPS", "n_gpus": 1, "steps": n,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8 QK^T (int32 acc) + fp16 PV (fp32 acc)",
+        "data": "synthetic (seeded numpy N(0,1) fp16, per-channel K offsets)",
+        "config": {"workload": "decode-causal-B8H32Hkv8Lq1Lk32768d128", **sh, "causal": True,
+                   "q_block_rows": 1, "kv_cache": "int8 K + fp16 V resident in HBM",
+                   "l2": "flushed before every timed step (256 MiB write)"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                     "frac": gbs / hbm, "traffic": None, "kernel": "sage_decode_kernel",
+                     "bytes_per_launch": int(nbytes),
+                     "peak_note": f"{peaks.get('source')} hbm_gbs (measured copy)"},
+        "gpu_launches": launches,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -442,8 +524,14 @@ def main():
                     help="rows per Q quantization block (finer than the 128-row tile)")
     ap.add_argument("--pv-accum", default="f32", choices=["f32", "f16"],
                     help="P V accumulator: fp32 (default) or fp16 as the article states")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decoding layout on one query token per head against a "
+                         "32768-token KV cache instead of the forward workloads")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)   # at least 3 untimed warm-up steps
+    if args.decode:
+        return run_decode_bench(args) if args.impl == "ours" else print(json.dumps(
+            {"impl": "reference", "unavailable": "the decode timing has no CPU reference arm"}))
     w = inputs.WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)

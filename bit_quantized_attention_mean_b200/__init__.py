@@ -10,9 +10,10 @@ Exported names mirror the C ABI:
     sage_quant_qk, sage_attn_fwd, sage_attn_fwd_prequant,
     sage_quant_qk_qblock, sage_attn_fwd_qblock, sage_attn_fwd_prequant_qblock,
     sage_attn_fwd_ex, sage_attn_fwd_prequant_ex,
+    sage_attn_decode, sage_attn_decode_prequant, sage_attn_decode_workspace_size,
     sage_quant_workspace_size, sage_attn_workspace_size,
     sage_check_device_status, sage_status_string, sage_last_launch_count
-plus two conveniences that allocate outputs: ``quant_qk`` and ``attention``.
+plus conveniences that allocate outputs: ``quant_qk``, ``attention`` and ``decode``.
 """
 from __future__ import annotations
 
@@ -43,4 +44,8 @@ from ._lib import (  # noqa: F401
     sage_status_string,
     quant_qk,
     attention,
+    decode,
+    sage_attn_decode,
+    sage_attn_decode_prequant,
+    sage_attn_decode_workspace_size,
 )

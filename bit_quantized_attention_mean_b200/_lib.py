@@ -33,6 +33,9 @@ SYMBOLS = (
     "sage_attn_fwd_qblock",
     "sage_attn_fwd_ex",
     "sage_attn_fwd_prequant_ex",
+    "sage_attn_decode_prequant",
+    "sage_attn_decode_workspace_size",
+    "sage_attn_decode",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
@@ -98,6 +101,12 @@ def load_library():
         lib.sage_attn_fwd_ex.restype = I
         lib.sage_attn_fwd_prequant_ex.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, U, P]
         lib.sage_attn_fwd_prequant_ex.restype = I
+        lib.sage_attn_decode_prequant.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, Z, P]
+        lib.sage_attn_decode_prequant.restype = I
+        lib.sage_attn_decode_workspace_size.argtypes = [I, I, I, I, I, I]
+        lib.sage_attn_decode_workspace_size.restype = Z
+        lib.sage_attn_decode.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+        lib.sage_attn_decode.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -288,6 +297,45 @@ def sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_bl
     _check(load_library().sage_attn_fwd_prequant_ex(*args, 1 if causal else 0,
                                                     int(q_block_rows), flags, _stream(stream)),
            "sage_attn_fwd_prequant_ex")
+
+
+def sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
+    return load_library().sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d)
+
+
+def sage_attn_decode_prequant(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_block_rows=128,
+                              workspace=None, stream=None):
+    """Few query tokens against a long key sequence, on pre-quantized Q/K
+    ((H / Hkv) * Lq <= 128)."""
+    _check_qbr(q_block_rows)
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
+    _check(load_library().sage_attn_decode_prequant(*args, 1 if causal else 0,
+                                                    int(q_block_rows), *_workspace(workspace),
+                                                    _stream(stream)),
+           "sage_attn_decode_prequant")
+
+
+def sage_attn_decode(q, k, v, out, causal, sm_scale, q_block_rows=128, stream=None):
+    """Quantization + sage_attn_decode_prequant on fp16 device tensors."""
+    import torch
+    _check_qbr(q_block_rows)
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    _check(lib.sage_attn_decode(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows),
+        _stream(stream)), "sage_attn_decode")
+
+
+def decode(q, k, v, causal=False, sm_scale=None, q_block_rows=128, stream=None):
+    """Allocate the output and run sage_attn_decode; returns the fp16 output."""
+    import torch
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    out = torch.empty_like(q)
+    sage_attn_decode(q, k, v, out, causal, sm_scale, q_block_rows, stream=stream)
+    return out
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20

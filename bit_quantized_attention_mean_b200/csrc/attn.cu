@@ -488,6 +488,10 @@ cudaError_t launch_wait_probe(int limit_ms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+cudaError_t device_status_address(int** p) {
+  return cudaGetSymbolAddress(reinterpret_cast<void**>(p), g_device_status);
+}
+
 cudaError_t read_and_clear_device_status(int* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, g_device_status, sizeof(int));
   if (e != cudaSuccess) return e;

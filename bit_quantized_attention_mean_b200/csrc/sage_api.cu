@@ -222,6 +222,91 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
+size_t sage_attn_decode_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
+  if (check_shape(B, H, Hkv, Lq, Lk, d) != SAGE_OK || (long long)(H / Hkv) * Lq > 128) return 0;
+  const sage::DecodePlan p = sage::decode_plan(B, H, Hkv, Lq, Lk, d);
+  return p.o_bytes + p.ml_bytes;
+}
+
+sage_status sage_attn_decode_prequant(const int8_t* q_i8, const int8_t* k_i8,
+                                      const float* q_scale, const float* k_scale, const void* v,
+                                      void* out, int B, int H, int Hkv, int Lq, int Lk, int d,
+                                      int causal, int q_block_rows, void* workspace,
+                                      size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if ((long long)(H / Hkv) * Lq > 128) return SAGE_ERR_UNSUPPORTED;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v || !out) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
+      !aligned16(q_scale) || !aligned16(k_scale))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  const sage::DecodePlan p = sage::decode_plan(B, H, Hkv, Lq, Lk, d);
+  const size_t need = p.o_bytes + p.ml_bytes;
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const bool own = !ws && need > 0;
+  if (own && cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  sage::DecodeArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
+                     static_cast<__half*>(out), need ? reinterpret_cast<float*>(ws) : nullptr,
+                     need ? reinterpret_cast<float2*>(ws + p.o_bytes) : nullptr,
+                     B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows};
+  int launches = 0;
+  cudaError_t e = sage::launch_decode(a, p, s, &launches);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_attn_decode(const void* q, const void* k, const void* v, void* out, int B, int H,
+                             int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
+                             int q_block_rows, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if ((long long)(H / Hkv) * Lq > 128) return SAGE_ERR_UNSUPPORTED;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const AttnWorkspace w = attn_workspace_layout(B, H, Hkv, Lq, Lk, d, q_block_rows);
+  const sage::DecodePlan p = sage::decode_plan(B, H, Hkv, Lq, Lk, d);
+  const size_t dec = p.o_bytes + p.ml_bytes;
+  char* ws = nullptr;
+  if (cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total + dec, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  int8_t* q_i8 = reinterpret_cast<int8_t*>(ws + w.q_i8);
+  int8_t* k_i8 = reinterpret_cast<int8_t*>(ws + w.k_i8);
+  float* q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+  float* k_scale = reinterpret_cast<float*>(ws + w.k_scale);
+  float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
+  sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
+                     q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
+                     fold_constant(sm_scale), q_block_rows};
+  int launches = 0;
+  cudaError_t e = sage::launch_quant(qa, s, &launches);
+  if (e == cudaSuccess) {
+    char* dws = ws + w.total;
+    sage::DecodeArgs da{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
+                        static_cast<__half*>(out), dec ? reinterpret_cast<float*>(dws) : nullptr,
+                        dec ? reinterpret_cast<float2*>(dws + p.o_bytes) : nullptr,
+                        B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows};
+    e = sage::launch_decode(da, p, s, &launches);
+  }
+  if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
 sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                void* out_host, int B, int H, int Hkv, int Lq, int Lk, int d,
                                int causal, float sm_scale, void* stream) {

@@ -42,6 +42,32 @@ struct AttnArgs {
 
 inline bool valid_q_block_rows(int r) { return r == 128 || r == 64 || r == 32 || r == 1; }
 
+// Few query tokens against a long key sequence: the query heads of a kv
+// group packed into one tile (rows = (H / Hkv) * Lq <= 128), keys split over
+// nsplit CTAs whose partial results a second kernel merges.
+struct DecodeArgs {
+  const int8_t* q_i8;
+  const int8_t* k_i8;
+  const float* q_scale;
+  const float* k_scale;
+  const __half* v;
+  __half* out;
+  float* o_part;    // [B*Hkv, nsplit, rows, d] partial outputs (nsplit > 1)
+  float2* ml_part;  // [B*Hkv, nsplit, rows] running max (base 2) and sum
+  int B, H, Hkv, Lq, Lk, d;
+  bool causal;
+  int q_block_rows;
+};
+
+struct DecodePlan {
+  int nsplit, split_tiles, rows;
+  size_t o_bytes, ml_bytes;  // scratch for the partials (0 when nsplit = 1)
+};
+
+DecodePlan decode_plan(int B, int H, int Hkv, int Lq, int Lk, int d);
+cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& p, cudaStream_t st,
+                          int* launches);
+
 size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d);
 
 // Each launcher adds the number of kernels it launched to *launches and
@@ -55,5 +81,6 @@ cudaError_t launch_wait_probe(int limit_ms, cudaStream_t st);
 
 // Device status word written by kernels whose bounded waits gave up.
 cudaError_t read_and_clear_device_status(int* value);
+cudaError_t device_status_address(int** p);
 
 }  // namespace sage

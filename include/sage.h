@@ -193,6 +193,46 @@ SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t 
                                    int causal, int q_block_rows, unsigned flags, void *stream);
 
 /*
+ * sage_attn_decode_prequant -- steps 3-5 for a few query tokens against a
+ * long key sequence (decoding against a KV cache): the same arithmetic as
+ * sage_attn_fwd_prequant, laid out for Lq << Lk.  The H / Hkv query heads of
+ * a kv head are packed into one 128-row tile, so each K/V tile is read from
+ * HBM once per kv head, and the keys are split over several CTAs whose
+ * partial results a second kernel merges (the merge is skipped when one
+ * split suffices).  Requires (H / Hkv) * Lq <= 128, else returns
+ * SAGE_ERR_UNSUPPORTED (use sage_attn_fwd_prequant_qblock).
+ *   q_i8, k_i8, q_scale, k_scale   as produced by sage_quant_qk_qblock with
+ *                                  the same q_block_rows
+ *   v, out, causal                 as sage_attn_fwd_prequant (bottom-right
+ *                                  causal alignment)
+ *   workspace, workspace_bytes     device scratch of at least
+ *                                  sage_attn_decode_workspace_size() bytes for
+ *                                  the partial results, or NULL/0 to let the
+ *                                  call allocate it with cudaMallocAsync on
+ *                                  `stream`.
+ * The article has no separate decoding kernel; this is the forward pass of
+ * its method for the GQA / long-context serving case it names.
+ */
+SAGE_API sage_status sage_attn_decode_prequant(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+/* Bytes of scratch sage_attn_decode_prequant needs (0 for unsupported shapes). */
+SAGE_API size_t sage_attn_decode_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
+
+/*
+ * sage_attn_decode -- quantization (sage_quant_qk_qblock) followed by
+ * sage_attn_decode_prequant on fp16 q, k, v; scratch allocated with
+ * cudaMallocAsync on `stream` and released on the same stream.
+ */
+SAGE_API sage_status sage_attn_decode(const void *q, const void *k, const void *v, void *out,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          int causal, float sm_scale, int q_block_rows, void *stream);
+
+/*
  * sage_attn_fwd_host -- sage_attn_fwd on HOST buffers, for callers whose data
  * lives in host memory.  q/k/v/out are host pointers with the layouts of
  * sage_attn_fwd (pinned memory gives asynchronous copies; pageable memory

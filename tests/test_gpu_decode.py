@@ -1,0 +1,108 @@
+"""GPU parity of the decoding layout (few query tokens, query heads of a kv
+group packed into one tile, keys split over CTAs and merged) against the CPU
+oracle, with the tolerances of the forward tests: quantized inputs are the
+same, and only the order of the softmax sums differs."""
+import ctypes
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import bit_quantized_attention_mean_b200 as sage
+from bit_quantized_attention_mean_b200 import inputs
+
+from test_gpu_parity import assert_close, cos, to_dev, torch_mod
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [
+    # B, H, Hkv, Lq, Lk, d, causal, q_block_rows
+    (1, 8, 2, 1, 1000, 128, False, 128),   # 4 heads per group, 16 splits of one tile
+    (2, 32, 8, 1, 4096, 128, True, 1),     # per-token Q scales
+    (1, 16, 16, 4, 777, 64, True, 1),      # 4 queries, bottom-right causal, ragged keys
+    (2, 8, 1, 16, 2048, 128, True, 32),    # 8 heads x 16 queries = a full 128-row tile
+    (4, 4, 4, 3, 130, 64, False, 128),     # three splits, ragged last tile
+    (64, 8, 8, 1, 256, 128, False, 128),   # many groups: one split, no merge
+    (1, 2, 2, 5, 3, 64, True, 1),          # fewer keys than queries: empty rows
+]
+
+
+def run_decode(q, k, v, causal, sm, qbr):
+    out = sage.decode(to_dev(q), to_dev(k), to_dev(v), causal, sm, q_block_rows=qbr)
+    sage.sage_check_device_status()
+    return out.cpu().numpy()
+
+
+@pytest.mark.parametrize("shape", SHAPES)
+def test_decode_against_oracle(shape):
+    B, H, Hkv, Lq, Lk, d, causal, qbr = shape
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=Lk + 7 * Lq, k_offset_sigma=2.0)
+    sm = float(np.float32(1 / math.sqrt(d)))
+    out = run_decode(q, k, v, causal, sm, qbr)
+    qk = oracle.quant_qk(q, k, sm, q_block_rows=qbr)
+    sim = oracle.attn_quant_sim(*qk[:4], v, causal, q_block_rows=qbr)
+    ref = oracle.attn_fp64(q, k, v, causal, sm)
+    assert_close(out, sim, ref, str(shape))
+
+
+def test_decode_matches_forward_layout():
+    torch = torch_mod()
+    q, k, v = inputs.make_custom(2, 16, 4, 2, 3000, 128, seed=91)
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    a = sage.decode(dq, dk, dv, True, 0.088, q_block_rows=1)
+    b = sage.attention(dq, dk, dv, True, 0.088, q_block_rows=1)
+    sage.sage_check_device_status()
+    a, b = a.cpu().numpy().astype(np.float64), b.cpu().numpy().astype(np.float64)
+    assert np.abs(a - b).max() < 2e-3 and cos(a, b) > 0.99999
+
+
+def test_prequant_with_caller_workspace():
+    torch = torch_mod()
+    B, H, Hkv, Lq, Lk, d = 1, 8, 2, 1, 5000, 128
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=92)
+    sm = 0.088
+    dq, dk, dv = to_dev(q), to_dev(k), to_dev(v)
+    qi, ki, qs, ks, km = sage.quant_qk(dq, dk, sm, q_block_rows=1)
+    need = sage.sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d)
+    assert need > 0
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    o1 = torch.empty_like(dq)
+    sage.sage_attn_decode_prequant(qi, ki, qs, ks, dv, o1, False, 1, workspace=ws)
+    o2 = torch.empty_like(dq)
+    sage.sage_attn_decode_prequant(qi, ki, qs, ks, dv, o2, False, 1)
+    o3 = sage.decode(dq, dk, dv, False, sm, q_block_rows=1)
+    sage.sage_check_device_status()
+    assert torch.equal(o1, o2) and torch.equal(o2, o3)
+
+
+def test_unsupported_and_invalid_decode_shapes():
+    torch = torch_mod()
+    lib = sage.load_library()
+    P = ctypes.c_void_p
+    s = P(torch.cuda.current_stream().cuda_stream)
+    q = torch.zeros((1, 16, 9, 64), dtype=torch.float16, device="cuda")   # 16 heads x 9 > 128
+    k = torch.zeros((1, 1, 256, 64), dtype=torch.float16, device="cuda")
+    out = torch.empty_like(q)
+    st = lib.sage_attn_decode(P(q.data_ptr()), P(k.data_ptr()), P(k.data_ptr()),
+                              P(out.data_ptr()), 1, 16, 1, 9, 256, 64, 0, 0.125, 128, s)
+    assert st == 2
+    assert lib.sage_attn_decode_workspace_size(1, 16, 1, 9, 256, 64) == 0
+    st = lib.sage_attn_decode(P(q.data_ptr()), P(k.data_ptr()), P(k.data_ptr()),
+                              P(out.data_ptr()), 1, 16, 1, 8, 256, 64, 0, 0.125, 7, s)
+    assert st == 1   # bad q_block_rows
+    sage.sage_check_device_status()
+
+
+def test_decode_full_size_sampled_rows():
+    """B=8, H=32, Hkv=8, one query token against 32768 keys (d = 128): the
+    serving shape the decode layout is for; every output row checked."""
+    B, H, Hkv, Lq, Lk, d = 8, 32, 8, 1, 32768, 128
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=93, k_offset_sigma=1.0)
+    sm = float(np.float32(1 / math.sqrt(d)))
+    out = run_decode(q, k, v, True, sm, 1).reshape(-1, d)
+    qk = oracle.quant_qk(q, k, sm, q_block_rows=1)
+    rows = np.arange(B * H * Lq, dtype=np.int64)
+    sim = oracle.attn_quant_sim(*qk[:4], v, True, rows=rows, q_block_rows=1)
+    ref = oracle.attn_fp64(q, k, v, True, sm, rows=rows)
+    assert_close(out, sim, ref, "decode B8 H32 Hkv8 Lq1 Lk32768 d128")
