@@ -55,8 +55,10 @@ INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "792aafd858761851", "workload": "llm-causal-B1H32L4096d128",
-               "bytes_per_launch": 68349184 + 6456576}
+NCU_TRAFFIC = {"attn_sha": "c4790aa86c5a578c", "workload": "llm-causal-B1H32L4096d128",
+               "bytes_per_launch": 69575168 + 4904192}
+# Same for the decoding kernel (decode.cu + PTX wrappers) on the --decode shape.
+DECODE_NCU_TRAFFIC = {"sha": "43151d8f92fa3db4", "bytes_per_launch": 805511168 + 3426304}
 
 
 def load_peaks():
@@ -67,6 +69,16 @@ def load_peaks():
         d["source"] = "measured"
         return d
     return dict(FALLBACK_PEAKS)
+
+
+def decode_source_hash():
+    """Hash of the decoding kernel's source and of the PTX wrappers."""
+    csrc = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc")
+    h = hashlib.sha256()
+    for name in ("decode.cu", "sm100_ptx.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def attn_source_hash():
@@ -499,7 +511,10 @@ def run_decode_bench(args):
                    "q_block_rows": 1, "kv_cache": "int8 K + fp16 V resident in HBM",
                    "l2": "flushed before every timed step (256 MiB write)"},
         "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                     "frac": gbs / hbm, "traffic": None, "kernel": "sage_decode_kernel",
+                     "frac": gbs / hbm,
+                     "traffic": (DECODE_NCU_TRAFFIC["bytes_per_launch"]
+                                 if DECODE_NCU_TRAFFIC["sha"] == decode_source_hash() else None),
+                     "kernel": "sage_decode_kernel",
                      "bytes_per_launch": int(nbytes),
                      "peak_note": f"{peaks.get('source')} hbm_gbs (measured copy)"},
         "gpu_launches": launches,
