@@ -14,6 +14,10 @@ Functions and the passages they follow (SageAttention article, method section):
                   in FP16, "对 P, V 采用 FP16 ..."
   attn_fp64       plain softmax(QK^T * sm_scale) V in fp64 (the accuracy
                   baseline the article compares against, "全精度 Attention")
+  e4m3_encode /   the FP8 (E4M3) format of the SageAttention2 description
+  e4m3_decode     ("将 P, V 量化至 FP8"), round to nearest even, saturating
+  quant_v_fp8     V to E4M3 with one scale per channel, stored channel-major
+  attn_fp8pv_sim  the forward pass with P and V in E4M3 for the P V product
 """
 from __future__ import annotations
 
@@ -72,6 +76,14 @@ def _load():
         lib.oracle_attn_quant_sim_blocks.restype = None
         lib.oracle_attn_fp64.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P, I64, P]
         lib.oracle_attn_fp64.restype = None
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = D
+        lib.oracle_quant_v_fp8.argtypes = [P, I, I, I, I, P, P]
+        lib.oracle_quant_v_fp8.restype = None
+        lib.oracle_attn_fp8pv_sim.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I, P, I64, P]
+        lib.oracle_attn_fp8pv_sim.restype = None
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = I
         _lib = lib
@@ -181,3 +193,46 @@ def attention(q, k, v, causal: bool, sm_scale: float, rows=None):
     Returns (out_f64, (q_i8, k_i8, q_scale, k_scale, k_mean))."""
     qk = quant_qk(q, k, sm_scale)
     return attn_quant_sim(qk[0], qk[1], qk[2], qk[3], v, causal, rows), qk
+
+
+def e4m3_encode(x: float) -> int:
+    return _load().oracle_e4m3_encode(float(x))
+
+
+def e4m3_decode(code: int) -> float:
+    return _load().oracle_e4m3_decode(int(code))
+
+
+def quant_v_fp8(v: np.ndarray):
+    """v: fp16 [B, Hkv, Lk, d] -> (v8t uint8 [B, Hkv, d, Lk], v_scale float32 [B, Hkv, d])."""
+    v = _c(v, np.float16)
+    B, Hkv, Lk, d = v.shape
+    v8t = np.empty((B, Hkv, d, Lk), dtype=np.uint8)
+    vs = np.empty((B, Hkv, d), dtype=np.float32)
+    _load().oracle_quant_v_fp8(_ptr(v), B, Hkv, Lk, d, _ptr(v8t), _ptr(vs))
+    return v8t, vs
+
+
+def attn_fp8pv_sim(q_i8, k_i8, q_scale, k_scale, v8t, v_scale, causal: bool, rows=None,
+                   q_block_rows: int = 128):
+    """Quantized forward pass with P and V in E4M3; float64 [n_rows, d] (or
+    [B, H, Lq, d] when rows is None)."""
+    q_i8 = _c(q_i8, np.int8)
+    k_i8 = _c(k_i8, np.int8)
+    q_scale = _c(q_scale, np.float32)
+    k_scale = _c(k_scale, np.float32)
+    v8t = _c(v8t, np.uint8)
+    v_scale = _c(v_scale, np.float32)
+    B, H, Lq, d = q_i8.shape
+    Hkv, Lk = k_i8.shape[1], k_i8.shape[2]
+    if rows is None:
+        out = np.empty((B, H, Lq, d), dtype=np.float64)
+        rp, n = None, 0
+    else:
+        rows = _c(np.asarray(rows, dtype=np.int64), np.int64)
+        out = np.empty((rows.shape[0], d), dtype=np.float64)
+        rp, n = _ptr(rows), rows.shape[0]
+    _load().oracle_attn_fp8pv_sim(_ptr(q_i8), _ptr(k_i8), _ptr(q_scale), _ptr(k_scale),
+                                  _ptr(v8t), _ptr(v_scale), B, H, Hkv, Lq, Lk, d,
+                                  1 if causal else 0, int(q_block_rows), rp, n, _ptr(out))
+    return out

@@ -335,6 +335,131 @@ void oracle_attn_fp64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
 }
 
+/* ------------------------------------------------------ FP8 (E4M3) P V */
+
+/* SageAttention2 as the pages describe it keeps P and V in FP8 (E4M3) for the
+ * P V product.  E4M3 here is the finite-only format with 1 sign bit, 4
+ * exponent bits (bias 7) and 3 mantissa bits: normals (1 + m/8) 2^(e-7) for
+ * e = 1..15 (e = 15, m = 7 is not a number), subnormals m 2^-9, largest
+ * finite value 448.  Conversion rounds to nearest, ties to even, and clamps
+ * magnitudes above 448 to 448 (saturating). */
+uint8_t oracle_e4m3_encode(float x)
+{
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0)
+        return sign | 0x7E;
+    if (a < 0.015625) {                       /* below 2^-6: subnormal grid 2^-9 */
+        double t = a * 512.0;                 /* exact */
+        double m = nearbyint(t);              /* ties to even (default rounding mode) */
+        return sign | (uint8_t)m;             /* m = 8 is the smallest normal, code 0x08 */
+    }
+    int e = 0;
+    double f = frexp(a, &e);                  /* a = f 2^e, f in [0.5, 1) */
+    int ex = e - 1;                           /* a = (2f) 2^ex, 2f in [1, 2) */
+    double m = nearbyint((2.0 * f - 1.0) * 8.0);
+    if (m == 8.0) { m = 0.0; ++ex; }
+    if (ex > 8 || (ex == 8 && m > 6.0))
+        return sign | 0x7E;
+    return sign | (uint8_t)(((ex + 7) << 3) | (int)m);
+}
+
+double oracle_e4m3_decode(uint8_t c)
+{
+    int e = (c >> 3) & 0xF, m = c & 7;
+    double v = e == 0 ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (c & 0x80) ? -v : v;
+}
+
+/* V -> E4M3 with one scale per channel over all Lk tokens of a (batch, kv
+ * head): a = max_t |V[t, c]|, r = fl32(448 / a), code = e4m3(fl32(V * r)),
+ * scale = fl32(a / 448); a zero channel gives codes 0 and scale 0.  The codes
+ * are stored channel-major, v8t [B, Hkv, d, Lk]. */
+void oracle_quant_v_fp8(const uint16_t *v, int B, int Hkv, int Lk, int d, uint8_t *v8t,
+                        float *v_scale)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t bc = 0; bc < (int64_t)B * Hkv * d; ++bc) {
+        int64_t bh = bc / d;
+        int c = (int)(bc % d);
+        const uint16_t *src = v + bh * Lk * d + c;
+        float a = 0.0f;
+        for (int t = 0; t < Lk; ++t) {
+            float x = (float)fabs(oracle_half_to_double(src[(int64_t)t * d]));
+            if (x > a) a = x;
+        }
+        float r = a > 0.0f ? 448.0f / a : 0.0f;
+        uint8_t *dst = v8t + (bh * d + c) * (int64_t)Lk;
+        for (int t = 0; t < Lk; ++t) {
+            float x = (float)oracle_half_to_double(src[(int64_t)t * d]) * r;
+            dst[t] = oracle_e4m3_encode(x);
+        }
+        v_scale[bh * d + c] = a > 0.0f ? a / 448.0f : 0.0f;
+    }
+}
+
+/* Quantized forward pass with P and V in E4M3: S, s and the exact row max as
+ * in oracle_attn_quant_sim; p = exp2(s - max) in fp64; P8 = e4m3(fl32(fl32(p)
+ * * 448)) (p <= 1 maps onto the E4M3 range); O = sum_j e4m3(P8)/448 *
+ * e4m3(V8[c][j]) * v_scale[c] / sum_j p (the row sum of the unquantized
+ * probabilities). */
+void oracle_attn_fp8pv_sim(const int8_t *q_i8, const int8_t *k_i8, const float *q_scale,
+                           const float *k_scale, const uint8_t *v8t, const float *v_scale,
+                           int B, int H, int Hkv, int Lq, int Lk, int d, int causal, int BQ,
+                           const int64_t *rows, int64_t n_rows, double *out)
+{
+    const int nqb = (Lq + BQ - 1) / BQ, nkb = (Lk + 63) / 64;
+    const int group = H / Hkv;
+    if (!rows)
+        n_rows = (int64_t)B * H * Lq;
+
+#pragma omp parallel
+    {
+        double *s = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+        double *pq = (double *)malloc(sizeof(double) * (size_t)(Lk > 0 ? Lk : 1));
+#pragma omp for schedule(dynamic, 4)
+        for (int64_t r = 0; r < n_rows; ++r) {
+            int64_t flat = rows ? rows[r] : r;
+            int i = (int)(flat % Lq);
+            int64_t bh = flat / Lq;
+            int b = (int)(bh / H), h = (int)(bh % H);
+            int64_t bhk = (int64_t)b * Hkv + h / group;
+            double *o = out + r * d;
+            for (int c = 0; c < d; ++c) o[c] = 0.0;
+            int64_t nvis = visible_keys(i, Lq, Lk, causal);
+            if (nvis == 0)
+                continue;
+            const int8_t *qi = q_i8 + (bh * Lq + i) * d;
+            double sq = (double)q_scale[bh * nqb + i / BQ];
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < nvis; ++j) {
+                const int8_t *kj = k_i8 + (bhk * Lk + j) * d;
+                int32_t acc = 0;
+                for (int c = 0; c < d; ++c)
+                    acc += (int32_t)qi[c] * (int32_t)kj[c];
+                s[j] = (double)acc * sq * (double)k_scale[bhk * nkb + j / 64];
+                if (s[j] > mx) mx = s[j];
+            }
+            double l = 0.0;
+            for (int64_t j = 0; j < nvis; ++j) {
+                double p = exp2(s[j] - mx);
+                l += p;
+                float p448 = (float)p * 448.0f;
+                pq[j] = oracle_e4m3_decode(oracle_e4m3_encode(p448)) / 448.0;
+            }
+            for (int c = 0; c < d; ++c) {
+                const uint8_t *vc = v8t + (bhk * d + c) * (int64_t)Lk;
+                double acc = 0.0;
+                for (int64_t j = 0; j < nvis; ++j)
+                    acc += pq[j] * oracle_e4m3_decode(vc[j]);
+                o[c] = acc * (double)v_scale[bhk * d + c] / l;
+            }
+        }
+        free(s);
+        free(pq);
+    }
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

@@ -480,3 +480,93 @@ def test_inputs_are_seeded_and_shaped():
     assert inputs.visible_pairs(1, 1, 4, 4, True) == 10
     assert inputs.visible_pairs(1, 1, 2, 4, True) == 7      # bottom-right: rows see 3, 4
     assert inputs.visible_pairs(1, 1, 4, 2, True) == 3      # rows see 0, 0, 1, 2
+
+
+# ------------------------------------------------------ FP8 (E4M3) P V
+
+def _torch_e4m3(values):
+    import torch
+    t = torch.tensor(np.asarray(values, dtype=np.float32))
+    return t.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_e4m3_decode_matches_torch_all_codes():
+    import torch
+    codes = [c for c in range(256) if c not in (0x7F, 0xFF)]     # the two NaN codes
+    want = torch.tensor(codes, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle.e4m3_decode(c) for c in codes])
+    assert np.array_equal(got, want.astype(np.float64))
+
+
+def test_e4m3_encode_matches_torch_rne_and_saturates():
+    """Round to nearest even against torch's float8_e4m3fn conversion on every
+    finite code, the midpoints between neighbouring codes (ties), points just
+    off the midpoints and random magnitudes; values above 448 saturate."""
+    import torch
+    finite = np.array(sorted({oracle.e4m3_decode(c) for c in range(0x7F)}))   # 0 .. 448
+    mids = (finite[:-1] + finite[1:]) / 2
+    off = np.concatenate([mids * (1 + 2.0 ** -20), mids * (1 - 2.0 ** -20)])
+    rng = np.random.default_rng(3)
+    rand = np.exp(rng.uniform(np.log(2.0 ** -12), np.log(448.0), size=4000))
+    xs = np.concatenate([finite, mids, off, rand]).astype(np.float32)
+    xs = np.concatenate([xs, -xs])
+    got = np.array([oracle.e4m3_encode(float(x)) for x in xs], dtype=np.uint8)
+    assert np.array_equal(got, _torch_e4m3(xs))
+    for big in (448.01, 464.0, 1e6):
+        assert oracle.e4m3_encode(big) == 0x7E and oracle.e4m3_encode(-big) == 0xFE
+
+
+def test_quant_v_fp8_properties():
+    rng = np.random.default_rng(8)
+    v = (rng.standard_normal((1, 2, 300, 64)) * 3).astype(np.float16)
+    v[0, 1, :, 5] = 0                                  # an all-zero channel
+    v8t, vs = oracle.quant_v_fp8(v)
+    assert v8t.shape == (1, 2, 64, 300) and vs.shape == (1, 2, 64)
+    dec = np.vectorize(oracle.e4m3_decode)(v8t)       # [B, Hkv, d, Lk]
+    vt = np.swapaxes(v.astype(np.float64), 2, 3)      # [B, Hkv, d, Lk]
+    amax = np.abs(vt).max(axis=3)
+    assert vs[0, 1, 5] == 0 and np.all(v8t[0, 1, 5] == 0)
+    nz = amax > 0
+    assert np.all(np.abs(dec).max(axis=3)[nz] == 448.0)
+    assert np.allclose(vs[nz], (amax / 448)[nz], rtol=2 ** -23)
+    # E4M3 keeps 3 mantissa bits: within half a unit in the last place of the
+    # scaled value (relative 2^-4 for normals, 2^-10 absolute below 2^-6)
+    scaled = vt * (448.0 / np.where(nz, amax, 1.0))[..., None]
+    err = np.abs(dec - scaled)
+    assert np.all(err <= np.maximum(np.abs(scaled) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-6))
+
+
+def test_fp8pv_sim_closed_forms():
+    """Equal scores give p = 1 for every visible key, which E4M3 holds
+    exactly (448), so the FP8 path returns the plain mean of the dequantized
+    V rows; causal row 0 returns the dequantized V row 0."""
+    B, H, L, d = 1, 2, 200, 64
+    q, k, v = inputs.make_custom(B, H, H, L, L, d, seed=44)
+    ke = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    sm = 1 / 8
+    qk = oracle.quant_qk(q, ke, sm)
+    v8t, vs = oracle.quant_v_fp8(v)
+    deq = np.swapaxes(np.vectorize(oracle.e4m3_decode)(v8t), 2, 3) * vs[:, :, None, :]
+    out = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, True)
+    exp = np.cumsum(deq, axis=2) / np.arange(1, L + 1)[None, None, :, None]
+    assert np.allclose(out, exp, rtol=1e-12, atol=1e-12)
+    out_nc = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, False)
+    assert np.allclose(out_nc, np.broadcast_to(deq.mean(axis=2, keepdims=True), out_nc.shape),
+                       rtol=1e-12, atol=1e-12)
+
+
+def test_fp8pv_sim_tracks_the_fp16_path_and_gqa():
+    q, k, v = inputs.make_custom(1, 4, 2, 256, 256, 64, seed=45)
+    sm = 1 / 8
+    qk = oracle.quant_qk(q, k, sm)
+    v8t, vs = oracle.quant_v_fp8(v)
+    f8 = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, True)
+    f16 = oracle.attn_quant_sim(*qk[:4], v, True)
+    a, b = f8.ravel(), f16.ravel()
+    assert a @ b / np.linalg.norm(a) / np.linalg.norm(b) > 0.999
+    assert not np.allclose(f8, f16)            # the FP8 rounding is really applied
+    # GQA: the same as repeating each kv head for its query heads
+    rep = lambda t: np.repeat(t, 2, axis=1)
+    qk2 = (qk[0], rep(qk[1]), qk[2], rep(qk[3]))
+    v8t2, vs2 = oracle.quant_v_fp8(rep(v))
+    assert np.array_equal(oracle.attn_fp8pv_sim(*qk2, v8t2, vs2, True), f8)
