@@ -288,6 +288,12 @@ def run_ours(args, w):
     k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
     ws = torch.empty(max(1, sage.sage_quant_workspace_size(B, Hkv, Lk, d)), dtype=torch.uint8,
                      device=dev)
+    fp8 = args.pv_accum == "fp8"
+    if fp8:
+        v8t = torch.empty((B, Hkv, d, -(-Lk // 64) * 64), dtype=torch.uint8, device=dev)
+        v_scale = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
+        ws8 = torch.empty(sage.sage_quant_v_fp8_workspace_size(B, Hkv, d), dtype=torch.uint8,
+                          device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     launches = 0
@@ -301,9 +307,15 @@ def run_ours(args, w):
             sage.sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, qbr,
                                       workspace=ws, stream=stream)
         launches += sage.sage_last_launch_count()
+        if fp8:   # V to E4M3 is part of the quantization step
+            sage.sage_quant_v_fp8(v, v8t, v_scale, workspace=ws8, stream=stream)
+            launches += sage.sage_last_launch_count()
         ev_mid = torch.cuda.Event(enable_timing=True)
         ev_mid.record(stream)
-        if args.pv_accum != "f32":
+        if fp8:
+            sage.sage_attn_fwd_prequant_fp8pv(q_i8, k_i8, q_scale, k_scale, v8t, v_scale, out,
+                                              w.causal, qbr, stream=stream)
+        elif args.pv_accum != "f32":
             sage.sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, w.causal, qbr,
                                            args.pv_accum, stream=stream)
         elif qbr == 128:
@@ -390,7 +402,8 @@ def run_ours(args, w):
         peaks = load_peaks()
         p16 = float(peaks["bf16_tflops"])
         p8 = INT8_OVER_FP16 * p16
-        t_roof_ms = (2.0 * d * w.pairs() / (p8 * 1e12) + 2.0 * d * w.pairs() / (p16 * 1e12)) * 1e3
+        p_pv = p8 if fp8 else p16   # FP8 P V runs at the 8-bit rate
+        t_roof_ms = (2.0 * d * w.pairs() / (p8 * 1e12) + 2.0 * d * w.pairs() / (p_pv * 1e12)) * 1e3
         peak_eff = ops / (t_roof_ms * 1e-3) / 1e12
         achieved = ops / (attn_avg_ms * 1e-3) / 1e12
         traffic = None
@@ -403,7 +416,8 @@ def run_ours(args, w):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": f"int8 QK^T (int32 acc) + fp16 PV ({args.pv_accum} acc)",
+            "dtype": ("int8 QK^T (int32 acc) + e4m3 PV (fp32 acc)" if fp8 else
+                      f"int8 QK^T (int32 acc) + fp16 PV ({args.pv_accum} acc)"),
             "data": "synthetic (seeded numpy N(0,1)/t4 fp16, per-channel K offsets)",
             "config": dict(w.describe(), q_block_rows=qbr, pv_accum=args.pv_accum,
                            l2="flushed before every timed step (256 MiB write)",
@@ -411,8 +425,9 @@ def run_ours(args, w):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
                          "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
                          "kernel": "sage_attn_fwd_kernel",
-                         "peak_note": (f"combined INT8/FP16 roofline: P_fp16 = {p16} TFLOP/s "
-                                       f"({peaks.get('source')} bf16 burst), P_int8 = "
+                         "peak_note": (f"combined roofline, QK at P_int8, PV at "
+                                       f"{'P_fp8 = P_int8' if fp8 else 'P_fp16'}: P_fp16 = {p16} "
+                                       f"TFLOP/s ({peaks.get('source')} bf16 burst), P_int8 = "
                                        f"{INT8_OVER_FP16} x P_fp16 (nominal ratio)")},
             "kernel_ms": {"attention": attn_avg_ms, "quant": quant_avg_ms},
             "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
@@ -537,8 +552,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-block-rows", type=int, default=128, choices=[128, 64, 32, 1],
                     help="rows per Q quantization block (finer than the 128-row tile)")
-    ap.add_argument("--pv-accum", default="f32", choices=["f32", "f16"],
-                    help="P V accumulator: fp32 (default) or fp16 as the article states")
+    ap.add_argument("--pv-accum", default="f32", choices=["f32", "f16", "fp8"],
+                    help="P V variant: fp16 P/V with fp32 sums (default), fp16 sums as the "
+                         "article states, or P and V in FP8 E4M3 (SageAttention2)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decoding layout on one query token per head against a "
                          "32768-token KV cache instead of the forward workloads")

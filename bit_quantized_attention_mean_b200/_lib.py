@@ -36,11 +36,15 @@ SYMBOLS = (
     "sage_attn_decode_prequant",
     "sage_attn_decode_workspace_size",
     "sage_attn_decode",
+    "sage_quant_v_fp8",
+    "sage_quant_v_fp8_workspace_size",
+    "sage_attn_fwd_prequant_fp8pv",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
 SAGE_PV_ACCUM_F16 = 1             # flag of the _ex calls: fp16 P V accumulator
-PV_ACCUM = {"f32": 0, "f16": SAGE_PV_ACCUM_F16}
+SAGE_PV_FP8 = 2                   # flag of sage_attn_fwd_ex: P and V in FP8 E4M3
+PV_ACCUM = {"f32": 0, "f16": SAGE_PV_ACCUM_F16, "fp8": SAGE_PV_FP8}
 
 STATUS = {0: "SAGE_OK", 1: "SAGE_ERR_INVALID_ARG", 2: "SAGE_ERR_UNSUPPORTED",
           3: "SAGE_ERR_CUDA", 4: "SAGE_ERR_TIMEOUT"}
@@ -107,6 +111,12 @@ def load_library():
         lib.sage_attn_decode_workspace_size.restype = Z
         lib.sage_attn_decode.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, P]
         lib.sage_attn_decode.restype = I
+        lib.sage_quant_v_fp8.argtypes = [P, P, P, I, I, I, I, P, Z, P]
+        lib.sage_quant_v_fp8.restype = I
+        lib.sage_quant_v_fp8_workspace_size.argtypes = [I, I, I]
+        lib.sage_quant_v_fp8_workspace_size.restype = Z
+        lib.sage_attn_fwd_prequant_fp8pv.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
+        lib.sage_attn_fwd_prequant_fp8pv.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -274,8 +284,10 @@ def _flags(pv_accum):
 
 def sage_attn_fwd_ex(q, k, v, out, causal, sm_scale, q_block_rows=128, pv_accum="f32",
                      stream=None):
-    """sage_attn_fwd with a Q block height and the P V accumulator ("f32",
-    the default, or "f16" as the SageAttention article states)."""
+    """sage_attn_fwd with a Q block height and the P V variant: "f32" (fp16 P
+    and V, fp32 sums; the default), "f16" (fp16 sums, as the SageAttention
+    article states) or "fp8" (P and V in E4M3, as its SageAttention2
+    description states)."""
     import torch
     _check_qbr(q_block_rows)
     flags = _flags(pv_accum)
@@ -290,9 +302,12 @@ def sage_attn_fwd_ex(q, k, v, out, causal, sm_scale, q_block_rows=128, pv_accum=
 
 def sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_block_rows=128,
                               pv_accum="f32", stream=None):
-    """sage_attn_fwd_prequant_qblock with the P V accumulator selectable."""
+    """sage_attn_fwd_prequant_qblock with the P V accumulator selectable
+    ("f32" or "f16"; FP8 P V takes E4M3 V: sage_attn_fwd_prequant_fp8pv)."""
     _check_qbr(q_block_rows)
     flags = _flags(pv_accum)
+    if flags == SAGE_PV_FP8:
+        raise ValueError("sage_attn_fwd_prequant_ex takes fp16 V; use sage_attn_fwd_prequant_fp8pv")
     args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
     _check(load_library().sage_attn_fwd_prequant_ex(*args, 1 if causal else 0,
                                                     int(q_block_rows), flags, _stream(stream)),
@@ -336,6 +351,50 @@ def decode(q, k, v, causal=False, sm_scale=None, q_block_rows=128, stream=None):
     out = torch.empty_like(q)
     sage_attn_decode(q, k, v, out, causal, sm_scale, q_block_rows, stream=stream)
     return out
+
+
+def sage_quant_v_fp8_workspace_size(B, Hkv, d) -> int:
+    return load_library().sage_quant_v_fp8_workspace_size(B, Hkv, d)
+
+
+def sage_quant_v_fp8(v, v8t, v_scale, workspace=None, stream=None):
+    """V fp16 [B, Hkv, Lk, d] -> E4M3 codes v8t uint8 [B, Hkv, d, 64*ceil(Lk/64)]
+    (channel-major) and per-channel scales v_scale fp32 [B, Hkv, d]."""
+    import torch
+    B, Hkv, Lk, d = v.shape
+    lkp = -(-Lk // 64) * 64
+    _check(load_library().sage_quant_v_fp8(
+        _dev(v, torch.float16, "v"), _dev(v8t, torch.uint8, "v8t", (B, Hkv, d, lkp)),
+        _dev(v_scale, torch.float32, "v_scale", (B, Hkv, d)), B, Hkv, Lk, d,
+        *_workspace(workspace), _stream(stream)), "sage_quant_v_fp8")
+
+
+def sage_attn_fwd_prequant_fp8pv(q_i8, k_i8, q_scale, k_scale, v8t, v_scale, out, causal,
+                                 q_block_rows=128, stream=None):
+    """Attention on pre-quantized Q/K with P and V in FP8 E4M3 (V from
+    sage_quant_v_fp8)."""
+    import torch
+    _check_qbr(q_block_rows)
+    B, H, Hkv, Lq, Lk, d = _dims(q_i8, k_i8)
+    nqb, nkb = -(-Lq // q_block_rows), -(-Lk // 64)
+    _check(load_library().sage_attn_fwd_prequant_fp8pv(
+        _dev(q_i8, torch.int8, "q_i8"), _dev(k_i8, torch.int8, "k_i8"),
+        _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
+        _dev(k_scale, torch.float32, "k_scale", (B, Hkv, nkb)),
+        _dev(v8t, torch.uint8, "v8t", (B, Hkv, d, nkb * 64)),
+        _dev(v_scale, torch.float32, "v_scale", (B, Hkv, d)),
+        _dev(out, torch.float16, "out", q_i8.shape), B, H, Hkv, Lq, Lk, d,
+        1 if causal else 0, int(q_block_rows), _stream(stream)), "sage_attn_fwd_prequant_fp8pv")
+
+
+def quant_v_fp8(v, stream=None):
+    """Allocate outputs and run sage_quant_v_fp8; returns (v8t, v_scale)."""
+    import torch
+    B, Hkv, Lk, d = v.shape
+    v8t = torch.empty((B, Hkv, d, -(-Lk // 64) * 64), dtype=torch.uint8, device=v.device)
+    vs = torch.empty((B, Hkv, d), dtype=torch.float32, device=v.device)
+    sage_quant_v_fp8(v, v8t, vs, stream=stream)
+    return v8t, vs
 
 
 NOALLOC_SCRATCH_BYTES = 64 << 20

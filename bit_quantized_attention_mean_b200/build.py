@@ -15,7 +15,7 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
-SOURCES = ["sage_api.cu", "quant.cu", "attn.cu", "noalloc.cu", "decode.cu"]
+SOURCES = ["sage_api.cu", "quant.cu", "attn.cu", "noalloc.cu", "decode.cu", "fp8.cu"]
 HEADERS = ["sage_internal.h", "sm100_ptx.cuh"]
 LIB = os.path.join(PKG, "libsage_b200.so")
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

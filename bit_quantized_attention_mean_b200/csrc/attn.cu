@@ -58,12 +58,17 @@ constexpr long long kGlobalOrderKVBytes = 112ll << 20;  // K/V total that stays 
 constexpr int BQ = 128;  // query rows per tile  (= Q quantization block)
 constexpr int BK = 64;   // key rows per tile    (= K quantization block)
 
-template <int D>
+// P V variants: fp16 P and V with fp32 sums (default), fp16 sums, or P and V
+// in E4M3 with fp32 sums.
+enum PvMode : int { kPvF32 = 0, kPvF16Acc = 1, kPvFp8 = 2 };
+
+template <int D, bool FP8V = false>
 struct AttnCfg {
   static constexpr int STAGES = 3;
   static constexpr int Q_BYTES = BQ * D;      // int8
   static constexpr int K_BYTES = BK * D;      // int8, per stage
-  static constexpr int V_BYTES = BK * D * 2;  // fp16, per stage
+  // per stage: fp16 V [64 keys x D], or E4M3 V^T [D channels x 64 keys]
+  static constexpr int V_BYTES = FP8V ? BK * D : BK * D * 2;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
@@ -113,13 +118,16 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __all_sync(0xffffffffu, ok);
 }
 
-template <int D, bool CAUSAL, bool F16ACC>
+template <int D, bool CAUSAL, int PV>
 __global__ void __launch_bounds__(192, 2)
 sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
-                     const float* __restrict__ k_scale, __half* __restrict__ out, int H, int Hkv,
-                     int Lq, int Lk, int nqt, int global_lpt, int qbr) {
-  using C = AttnCfg<D>;
+                     const float* __restrict__ k_scale, const float* __restrict__ v_scale,
+                     __half* __restrict__ out, int H, int Hkv, int Lq, int Lk, int nqt,
+                     int global_lpt, int qbr) {
+  constexpr bool F16ACC = PV == kPvF16Acc;
+  constexpr bool FP8V = PV == kPvFp8;
+  using C = AttnCfg<D, FP8V>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment of the shared-window address (swizzle atoms)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -190,10 +198,16 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tma_load_3d_hint(smem + C::OFF_K + s * C::K_BYTES, &tm_k, &bars[C::B_K_FULL + s], 0,
                          j * BK, bhk, keep);
         mbar_arrive_expect_tx(&bars[C::B_V_FULL + s], C::V_BYTES);
+        if constexpr (FP8V) {
+          // E4M3 V^T tile: D channel rows of 64 keys (64-byte swizzle)
+          tma_load_3d_hint(smem + C::OFF_V + s * C::V_BYTES, &tm_v, &bars[C::B_V_FULL + s],
+                           j * BK, 0, bhk, keep);
+        } else {
 #pragma unroll
-        for (int cc = 0; cc < D / 64; ++cc)
-          tma_load_3d_hint(smem + C::OFF_V + s * C::V_BYTES + cc * (BK * 128), &tm_v,
-                           &bars[C::B_V_FULL + s], cc * 64, j * BK, bhk, keep);
+          for (int cc = 0; cc < D / 64; ++cc)
+            tma_load_3d_hint(smem + C::OFF_V + s * C::V_BYTES + cc * (BK * 128), &tm_v,
+                             &bars[C::B_V_FULL + s], cc * 64, j * BK, bhk, keep);
+        }
         issued = j + 1;
       }
       // nothing may still be landing in shared memory when the CTA exits
@@ -208,7 +222,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     // ---------------------------------------------------------- MMA issuer
     if (lane == 0 && nkt > 0) {
       constexpr uint32_t idesc_qk = make_idesc_i8(BQ, BK);
-      constexpr uint32_t idesc_pv = make_idesc_f16(BQ, D, /*b_mn_major=*/true, F16ACC);
+      constexpr uint32_t idesc_pv =
+          FP8V ? make_idesc_f8(BQ, D) : make_idesc_f16(BQ, D, /*b_mn_major=*/true, F16ACC);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q);
       auto issue_pv = [&](int jj) -> bool {
         const int bb = jj & 1, ss = jj % C::STAGES;
@@ -220,14 +235,25 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tc_fence_after_sync();
         const uint32_t sV = smem_u32(smem + C::OFF_V + ss * C::V_BYTES);
         const uint32_t p_tmem = tmem + C::S_COL + 64u * bb;
+        if constexpr (FP8V) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          // V tile: D/64 chunks of [64 keys x 128 B] (128B swizzle), MN-major
-          // B operand; LBO = chunk stride, SBO = 8 key rows; 16 keys per MMA.
-          const uint64_t bdesc =
-              make_smem_desc(sV + kk * 16 * 128, BK * 128, 1024, kSwizzle128B);
-          umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8, bdesc, idesc_pv,
-                      (jj > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // V^T tile: K-major B operand, rows of 64 keys (64B swizzle), 8-row
+            // groups 512 B apart; 32 keys per MMA; P: 4 keys per column
+            const uint64_t bdesc = make_smem_desc(sV + kk * 32, 16, 512, kSwizzle64B);
+            umma_f8_ts(tmem + C::O_COL, p_tmem + kk * 8, bdesc, idesc_pv,
+                       (jj > 0 || kk > 0) ? 1u : 0u);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            // V tile: D/64 chunks of [64 keys x 128 B] (128B swizzle), MN-major
+            // B operand; LBO = chunk stride, SBO = 8 key rows; 16 keys per MMA.
+            const uint64_t bdesc =
+                make_smem_desc(sV + kk * 16 * 128, BK * 128, 1024, kSwizzle128B);
+            umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8, bdesc, idesc_pv,
+                        (jj > 0 || kk > 0) ? 1u : 0u);
+          }
         }
         umma_commit(&bars[C::B_KV_EMPTY + ss]);
         umma_commit(&bars[C::B_O_DONE]);
@@ -345,10 +371,18 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           p1 = k + 1 < vis ? p1 : 0.f;
         }
         lsum += p0 + p1;
-        pk[k >> 1] = pack_half2(p0, p1);
+        if constexpr (FP8V) {
+          // P <= 2^8 (lazy max), so P * 1.75 <= 448 fits E4M3; 4 keys a column
+          const uint32_t e = pack_e4m3x2(p0 * 1.75f, p1 * 1.75f);
+          pk[k >> 2] = (k & 2) ? (pk[k >> 2] | (e << 16)) : e;
+        } else {
+          pk[k >> 1] = pack_half2(p0, p1);
+        }
       }
       l_run += lsum;
-      tmem_st32(s_tmem, pk);  // P (fp16 pairs) over the consumed scores
+      // P over the consumed scores
+      if constexpr (FP8V) tmem_st16(s_tmem, pk);
+      else tmem_st32(s_tmem, pk);
       tc_fence_before_sync();
       mbar_arrive(&bars[C::B_P_FULL + bb]);
     }
@@ -371,9 +405,20 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
         uint32_t hv[16];
+        if constexpr (FP8V) {
+          // undo the per-channel V scale and the 1.75 of P
+          const float* vs = v_scale + (size_t)bhk * D + cc * 32;
+          const float s8 = inv * (1.0f / 1.75f);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          hv[i] = pack_half2(acc_value<F16ACC>(o[2 * i]) * inv, acc_value<F16ACC>(o[2 * i + 1]) * inv);
+          for (int i = 0; i < 16; ++i)
+            hv[i] = pack_half2(__uint_as_float(o[2 * i]) * (__ldg(vs + 2 * i) * s8),
+                               __uint_as_float(o[2 * i + 1]) * (__ldg(vs + 2 * i + 1) * s8));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            hv[i] = pack_half2(acc_value<F16ACC>(o[2 * i]) * inv,
+                               acc_value<F16ACC>(o[2 * i + 1]) * inv);
+        }
         if (qrow < Lq) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll
@@ -422,10 +467,10 @@ static bool make_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType 
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, bool CAUSAL, bool F16ACC>
+template <int D, bool CAUSAL, int PV>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launches) {
-  using C = AttnCfg<D>;
-  auto kern = sage_attn_fwd_kernel<D, CAUSAL, F16ACC>;
+  using C = AttnCfg<D, PV == kPvFp8>;
+  auto kern = sage_attn_fwd_kernel<D, CAUSAL, PV>;
   // per device context; cheap enough to repeat on every launch
   cudaError_t attr_err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -438,34 +483,39 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launch
                    BQ, qk_sw) ||
       !make_map_3d(&tk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, D, a.Lk, (uint64_t)a.B * a.Hkv,
                    D, BK, qk_sw) ||
-      !make_map_3d(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, a.Lk, (uint64_t)a.B * a.Hkv,
-                   64, BK, CU_TENSOR_MAP_SWIZZLE_128B))
+      !(PV == kPvFp8
+            ? make_map_3d(&tv, a.v8t, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1,
+                          (uint64_t)(a.Lk + BK - 1) / BK * BK, D, (uint64_t)a.B * a.Hkv, BK, D,
+                          CU_TENSOR_MAP_SWIZZLE_64B)
+            : make_map_3d(&tv, a.v, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, D, a.Lk,
+                          (uint64_t)a.B * a.Hkv, 64, BK, CU_TENSOR_MAP_SWIZZLE_128B)))
     return cudaErrorInvalidValue;
 
   const int nqt = (a.Lq + BQ - 1) / BQ;
   const long long grid = (long long)a.B * a.H * nqt;
-  const long long kv_bytes = (long long)a.B * a.Hkv * a.Lk * D * 3;  // int8 K + fp16 V
+  const long long kv_bytes = (long long)a.B * a.Hkv * a.Lk * D * (PV == kPvFp8 ? 2 : 3);
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.out, a.H,
-                                                   a.Hkv, a.Lq, a.Lk, nqt,
+  kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.v_scale,
+                                                   a.out, a.H, a.Hkv, a.Lq, a.Lk, nqt,
                                                    kv_bytes <= kGlobalOrderKVBytes ? 1 : 0,
                                                    a.q_block_rows);
   *launches += 1;
   return cudaGetLastError();
 }
 
-template <bool F16ACC>
-static cudaError_t launch_attn_acc(const AttnArgs& a, cudaStream_t st, int* launches) {
+template <int PV>
+static cudaError_t launch_attn_pv(const AttnArgs& a, cudaStream_t st, int* launches) {
   if (a.d == 128)
-    return a.causal ? launch_attn_t<128, true, F16ACC>(a, st, launches)
-                    : launch_attn_t<128, false, F16ACC>(a, st, launches);
-  return a.causal ? launch_attn_t<64, true, F16ACC>(a, st, launches)
-                  : launch_attn_t<64, false, F16ACC>(a, st, launches);
+    return a.causal ? launch_attn_t<128, true, PV>(a, st, launches)
+                    : launch_attn_t<128, false, PV>(a, st, launches);
+  return a.causal ? launch_attn_t<64, true, PV>(a, st, launches)
+                  : launch_attn_t<64, false, PV>(a, st, launches);
 }
 
 cudaError_t launch_attn(const AttnArgs& a, cudaStream_t st, int* launches) {
-  return a.pv_f16_accum ? launch_attn_acc<true>(a, st, launches)
-                        : launch_attn_acc<false>(a, st, launches);
+  if (a.pv_fp8) return launch_attn_pv<kPvFp8>(a, st, launches);
+  return a.pv_f16_accum ? launch_attn_pv<kPvF16Acc>(a, st, launches)
+                        : launch_attn_pv<kPvF32>(a, st, launches);
 }
 
 // One warp waits on an mbarrier that nothing ever completes, through the

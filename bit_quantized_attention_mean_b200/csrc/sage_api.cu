@@ -43,6 +43,13 @@ float fold_constant(float sm_scale) {
 
 size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
+// Accepted flag words of the _ex calls: 0, SAGE_PV_ACCUM_F16 or SAGE_PV_FP8.
+bool valid_flags(unsigned f) { return f == 0u || f == SAGE_PV_ACCUM_F16 || f == SAGE_PV_FP8; }
+
+size_t v8t_bytes(int B, int Hkv, int Lk, int d) {
+  return (size_t)B * Hkv * d * (size_t)((Lk + 63) / 64 * 64);
+}
+
 struct AttnWorkspace {
   size_t q_i8, k_i8, q_scale, k_scale, k_mean, part, total;
 };
@@ -151,7 +158,7 @@ sage_status sage_attn_fwd_prequant_ex(const int8_t* q_i8, const int8_t* k_i8,
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
-  if ((flags & ~(unsigned)SAGE_PV_ACCUM_F16) != 0u) return SAGE_ERR_INVALID_ARG;
+  if (!valid_flags(flags) || flags == SAGE_PV_FP8) return SAGE_ERR_INVALID_ARG;
   if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
       !aligned16(q_scale) || !aligned16(k_scale))
@@ -188,7 +195,7 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
-  if ((flags & ~(unsigned)SAGE_PV_ACCUM_F16) != 0u) return SAGE_ERR_INVALID_ARG;
+  if (!valid_flags(flags)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return SAGE_ERR_INVALID_ARG;
@@ -198,8 +205,13 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const AttnWorkspace w = attn_workspace_layout(B, H, Hkv, Lq, Lk, d, q_block_rows);
+  const bool fp8 = flags == SAGE_PV_FP8;
+  // E4M3 V^T, its channel scales and the maxima scratch after the common part
+  const size_t v8_off = w.total, vs_off = v8_off + round_up(v8t_bytes(B, Hkv, Lk, d));
+  const size_t vm_off = vs_off + round_up((size_t)B * Hkv * d * 4);
+  const size_t total = fp8 ? vm_off + sage::quant_v_fp8_workspace_bytes(B, Hkv, d) : w.total;
   char* ws = nullptr;
-  if (cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, s) != cudaSuccess)
+  if (cudaMallocAsync(reinterpret_cast<void**>(&ws), total, s) != cudaSuccess)
     return SAGE_ERR_CUDA;
   int8_t* q_i8 = reinterpret_cast<int8_t*>(ws + w.q_i8);
   int8_t* k_i8 = reinterpret_cast<int8_t*>(ws + w.k_i8);
@@ -211,10 +223,20 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
                      fold_constant(sm_scale), q_block_rows};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
+  uint8_t* v8t = reinterpret_cast<uint8_t*>(ws + v8_off);
+  float* v_scale = reinterpret_cast<float*>(ws + vs_off);
+  if (e == cudaSuccess && fp8)
+    e = sage::launch_quant_v_fp8(static_cast<const __half*>(v), v8t, v_scale, ws + vm_off, B, Hkv,
+                                 Lk, d, s, &launches);
   if (e == cudaSuccess) {
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                       static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,
-                      q_block_rows, (flags & SAGE_PV_ACCUM_F16) != 0u};
+                      q_block_rows, flags == SAGE_PV_ACCUM_F16};
+    if (fp8) {
+      aa.pv_fp8 = true;
+      aa.v8t = v8t;
+      aa.v_scale = v_scale;
+    }
     e = sage::launch_attn(aa, s, &launches);
   }
   if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
@@ -303,6 +325,60 @@ sage_status sage_attn_decode(const void* q, const void* k, const void* v, void* 
     e = sage::launch_decode(da, p, s, &launches);
   }
   if (cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+size_t sage_quant_v_fp8_workspace_size(int B, int Hkv, int d) {
+  if (B < 1 || Hkv < 1 || (d != 64 && d != 128)) return 0;
+  return sage::quant_v_fp8_workspace_bytes(B, Hkv, d);
+}
+
+sage_status sage_quant_v_fp8(const void* v, uint8_t* v8t, float* v_scale, int B, int Hkv, int Lk,
+                             int d, void* workspace, size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, Hkv, Hkv, 1, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!v || !v8t || !v_scale) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(v) || !aligned16(v8t) || !aligned16(v_scale)) return SAGE_ERR_INVALID_ARG;
+  const size_t need = sage::quant_v_fp8_workspace_bytes(B, Hkv, d);
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  const bool own = !ws;
+  if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  int launches = 0;
+  cudaError_t e = sage::launch_quant_v_fp8(static_cast<const __half*>(v), v8t, v_scale, ws, B,
+                                           Hkv, Lk, d, s, &launches);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
+sage_status sage_attn_fwd_prequant_fp8pv(const int8_t* q_i8, const int8_t* k_i8,
+                                         const float* q_scale, const float* k_scale,
+                                         const uint8_t* v8t, const float* v_scale, void* out,
+                                         int B, int H, int Hkv, int Lq, int Lk, int d, int causal,
+                                         int q_block_rows, void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if (!q_i8 || !k_i8 || !q_scale || !k_scale || !v8t || !v_scale || !out)
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v8t) || !aligned16(out) ||
+      !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(v_scale))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  sage::AttnArgs a{q_i8, k_i8, q_scale, k_scale, nullptr, static_cast<__half*>(out), B, H, Hkv,
+                   Lq, Lk, d, causal == 1, q_block_rows, false};
+  a.pv_fp8 = true;
+  a.v8t = v8t;
+  a.v_scale = v_scale;
+  int launches = 0;
+  cudaError_t e = sage::launch_attn(a, static_cast<cudaStream_t>(stream), &launches);
   g_last_launches = launches;
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }

@@ -38,7 +38,14 @@ struct AttnArgs {
   bool causal;
   int q_block_rows;   // rows per q_scale entry: 128, 64, 32 or 1
   bool pv_f16_accum;  // accumulate P V in fp16 (else fp32)
+  bool pv_fp8 = false;            // P and V in E4M3 (v8t, v_scale below; v unused)
+  const uint8_t* v8t = nullptr;   // E4M3 V^T [B, Hkv, d, 64 * ceil(Lk / 64)]
+  const float* v_scale = nullptr; // [B, Hkv, d]
 };
+
+size_t quant_v_fp8_workspace_bytes(int B, int Hkv, int d);
+cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8t, float* v_scale, void* workspace,
+                               int B, int Hkv, int Lk, int d, cudaStream_t st, int* launches);
 
 inline bool valid_q_block_rows(int r) { return r == 128 || r == 64 || r == 32 || r == 1; }
 

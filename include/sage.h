@@ -63,6 +63,7 @@ typedef enum {
 
 /* Flags of the _ex entry points. */
 #define SAGE_PV_ACCUM_F16 1u  /* accumulate P V in fp16 (the article's choice) */
+#define SAGE_PV_FP8 2u        /* P and V in FP8 E4M3, fp32 sums (SageAttention2) */
 
 /*
  * sage_quant_qk -- steps 1-2: smoothing of K and per-block INT8 quantization.
@@ -179,8 +180,13 @@ SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const vo
  * row max is kept exact (O is rescaled whenever it grows), so P <= 1 and, as
  * the article argues, the sums stay within the fp16 range; the result is
  * less accurate than the fp32 default (the error grows with Lk) and no
- * faster on this GPU.  flags = 0 is identical to the _qblock calls.  Any
- * other bit returns SAGE_ERR_INVALID_ARG.
+ * faster on this GPU.  SAGE_PV_FP8 (sage_attn_fwd_ex only) quantizes V to
+ * E4M3 per channel (sage_quant_v_fp8) and P to E4M3 and runs P V on the FP8
+ * tensor-core path with fp32 sums, as the SageAttention2 description on the
+ * same pages states ("将 P, V 量化至 FP8").  flags = 0 is identical to the
+ * _qblock calls.  Any other value, both bits together, or SAGE_PV_FP8 given
+ * to sage_attn_fwd_prequant_ex (which takes fp16 V; use
+ * sage_attn_fwd_prequant_fp8pv) returns SAGE_ERR_INVALID_ARG.
  */
 SAGE_API sage_status sage_attn_fwd_ex(const void *q, const void *k, const void *v, void *out,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
@@ -191,6 +197,36 @@ SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t 
                                    const void *v, void *out,
                                    int B, int H, int Hkv, int Lq, int Lk, int d,
                                    int causal, int q_block_rows, unsigned flags, void *stream);
+
+/*
+ * sage_quant_v_fp8 -- V to FP8 E4M3 with one scale per channel over all Lk
+ * tokens of a (batch, kv head): a = max_t |V[t, c]|, r = fl32(448 / a),
+ * code = e4m3(fl32(V * r)) (round to nearest even, saturating at 448),
+ * scale = fl32(a / 448); a zero channel gives codes 0 and scale 0.
+ *   v        fp16 [B, Hkv, Lk, d]                      (in)
+ *   v8t      uint8 [B, Hkv, d, Lkp], Lkp = 64*ceil(Lk/64) (out) E4M3 codes,
+ *            channel-major (keys contiguous); positions >= Lk hold 0
+ *   v_scale  fp32 [B, Hkv, d]                          (out)
+ *   workspace: sage_quant_v_fp8_workspace_size() bytes or NULL/0 (allocated
+ *   with cudaMallocAsync on `stream`).
+ */
+SAGE_API sage_status sage_quant_v_fp8(const void *v, uint8_t *v8t, float *v_scale,
+                                      int B, int Hkv, int Lk, int d,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+SAGE_API size_t sage_quant_v_fp8_workspace_size(int B, int Hkv, int d);
+
+/*
+ * sage_attn_fwd_prequant_fp8pv -- steps 3-5 with P and V in FP8 E4M3: V from
+ * sage_quant_v_fp8 (v8t, v_scale), P = e4m3(1.75 * p) with p relative to the
+ * running row max (p <= 2^8), P V on the tensor core's FP8 path with fp32
+ * sums, the row sum taken over the unquantized p.  Other arguments as
+ * sage_attn_fwd_prequant_qblock.
+ */
+SAGE_API sage_status sage_attn_fwd_prequant_fp8pv(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const uint8_t *v8t, const float *v_scale, void *out,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows, void *stream);
 
 /*
  * sage_attn_decode_prequant -- steps 3-5 for a few query tokens against a
