@@ -4,6 +4,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <mutex>
 
 #include "../../include/sage.h"
 #include "sage_internal.h"
@@ -48,6 +49,25 @@ bool valid_flags(unsigned f) { return f == 0u || f == SAGE_PV_ACCUM_F16 || f == 
 
 size_t v8t_bytes(int B, int Hkv, int Lk, int d) {
   return (size_t)B * Hkv * d * (size_t)((Lk + 63) / 64 * 64);
+}
+
+constexpr int kMaxDevices = 64;
+constexpr int kHostChunks = 8;  // chunks of (batch, kv head) groups in the host-buffer call
+
+// Three non-blocking side streams per device for the host-buffer call (copy
+// in, compute, copy out), created on first use and kept for the life of the
+// process.
+cudaStream_t* side_streams(int dev) {
+  static cudaStream_t streams[kMaxDevices][3];
+  static std::once_flag once[kMaxDevices];
+  static bool ok[kMaxDevices];
+  std::call_once(once[dev], [dev] {
+    ok[dev] = true;
+    for (int i = 0; i < 3; ++i)
+      ok[dev] = ok[dev] &&
+                cudaStreamCreateWithFlags(&streams[dev][i], cudaStreamNonBlocking) == cudaSuccess;
+  });
+  return ok[dev] ? streams[dev] : nullptr;
 }
 
 struct AttnWorkspace {
@@ -393,29 +413,104 @@ sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const voi
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
   if ((st = check_device()) != SAGE_OK) return st;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SAGE_ERR_CUDA;
+  cudaStream_t* side = side_streams(dev);
+  if (!side) return SAGE_ERR_CUDA;
 
+  // Every (batch, kv head) group is independent: its K mean, its blocks and
+  // its query heads.  Groups are processed in chunks through a three-stage
+  // pipeline on side streams: copy-in (all host->device copies back to back),
+  // compute (quantization + attention of chunk i once its copies are in) and
+  // copy-out (chunk i's output once computed), so the copy engines stay busy
+  // while the kernels run.  Query heads of groups [g0, g1) are the flat heads
+  // [g0 G, g1 G) and kv heads are [g0, g1), both contiguous, so a chunk is the
+  // problem B = 1, H = (g1 - g0) G, Hkv = g1 - g0.
+  const int G = H / Hkv;
+  const int groups = B * Hkv;
+  const int nchunk = groups < kHostChunks ? groups : kHostChunks;
+  const int per = (groups + nchunk - 1) / nchunk;
+  const size_t qh = (size_t)Lq * d * 2, kh = (size_t)Lk * d * 2;  // bytes per head
+  const size_t qb = (size_t)B * H * qh, kb = (size_t)B * Hkv * kh;
+  const AttnWorkspace w = attn_workspace_layout(1, per * G, per, Lq, Lk, d, SAGE_Q_BLOCK);
+  const size_t total = round_up(qb) * 2 + round_up(kb) * 2 + w.total;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t qb = (size_t)B * H * Lq * d * 2, kb = (size_t)B * Hkv * Lk * d * 2;
   char* buf = nullptr;
-  const size_t total = round_up(qb) * 2 + round_up(kb) * 2;
   if (cudaMallocAsync(reinterpret_cast<void**>(&buf), total, s) != cudaSuccess) return SAGE_ERR_CUDA;
   char* dq = buf;
   char* dout = dq + round_up(qb);
   char* dk = dout + round_up(qb);
   char* dv = dk + round_up(kb);
-  cudaError_t e = cudaMemcpyAsync(dq, q_host, qb, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dk, k_host, kb, cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess) e = cudaMemcpyAsync(dv, v_host, kb, cudaMemcpyHostToDevice, s);
-  int launches = 0;
-  if (e == cudaSuccess) {
-    st = sage_attn_fwd(dq, dk, dv, dout, B, H, Hkv, Lq, Lk, d, causal, sm_scale, stream);
-    launches = g_last_launches;
-    if (st != SAGE_OK) e = cudaErrorUnknown;
+  char* ws = dv + round_up(kb);
+  // events: [0, nchunk) copies in, [nchunk, 2 nchunk) computed, then start
+  // and the three stage ends
+  const int nev = 2 * nchunk + 4;
+  cudaEvent_t ev[2 * kHostChunks + 4];
+  int made = 0;
+  cudaError_t e = cudaSuccess;
+  for (; made < nev && e == cudaSuccess; ++made)
+    e = cudaEventCreateWithFlags(&ev[made], cudaEventDisableTiming);
+  if (e != cudaSuccess) {
+    for (int j = 0; j < made - 1; ++j) cudaEventDestroy(ev[j]);
+    cudaFreeAsync(buf, s);
+    return SAGE_ERR_CUDA;
   }
-  if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, dout, qb, cudaMemcpyDeviceToHost, s);
+  cudaEvent_t* ev_in = ev;
+  cudaEvent_t* ev_done = ev + nchunk;
+  cudaEvent_t ev_start = ev[2 * nchunk];
+  e = cudaEventRecord(ev_start, s);  // the buffer exists on `stream` from here
+  for (int i = 0; i < 3 && e == cudaSuccess; ++i) e = cudaStreamWaitEvent(side[i], ev_start, 0);
+  cudaStream_t cin = side[0], comp = side[1], cout = side[2];
+  const float c = fold_constant(sm_scale);
+  int launches = 0;
+  for (int ci = 0; ci < nchunk && e == cudaSuccess; ++ci) {
+    const int g0 = ci * per, g1 = g0 + per < groups ? g0 + per : groups;
+    const int n = g1 > g0 ? g1 - g0 : 0;
+    const size_t qo = (size_t)g0 * G * qh, ko = (size_t)g0 * kh;
+    if (n > 0) {
+      e = cudaMemcpyAsync(dk + ko, static_cast<const char*>(k_host) + ko, n * kh,
+                          cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dq + qo, static_cast<const char*>(q_host) + qo, n * G * qh,
+                            cudaMemcpyHostToDevice, cin);
+      if (e == cudaSuccess)
+        e = cudaMemcpyAsync(dv + ko, static_cast<const char*>(v_host) + ko, n * kh,
+                            cudaMemcpyHostToDevice, cin);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[ci], cin);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(comp, ev_in[ci], 0);
+    if (e == cudaSuccess && n > 0) {
+      int8_t* q_i8 = reinterpret_cast<int8_t*>(ws + w.q_i8);
+      int8_t* k_i8 = reinterpret_cast<int8_t*>(ws + w.k_i8);
+      float* q_scale = reinterpret_cast<float*>(ws + w.q_scale);
+      float* k_scale = reinterpret_cast<float*>(ws + w.k_scale);
+      float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
+      sage::QuantArgs qa{reinterpret_cast<const __half*>(dq + qo),
+                         reinterpret_cast<const __half*>(dk + ko), q_i8, k_i8, q_scale, k_scale,
+                         k_mean, ws + w.part, 1, n * G, n, Lq, Lk, d, c, SAGE_Q_BLOCK};
+      e = sage::launch_quant(qa, comp, &launches);
+      if (e == cudaSuccess) {
+        sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, reinterpret_cast<const __half*>(dv + ko),
+                          reinterpret_cast<__half*>(dout + qo), 1, n * G, n, Lq, Lk, d,
+                          causal == 1, SAGE_Q_BLOCK, false};
+        e = sage::launch_attn(aa, comp, &launches);
+      }
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev_done[ci], comp);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(cout, ev_done[ci], 0);
+    if (e == cudaSuccess && n > 0)
+      e = cudaMemcpyAsync(static_cast<char*>(out_host) + qo, dout + qo, n * G * qh,
+                          cudaMemcpyDeviceToHost, cout);
+  }
+  // `stream` resumes after the three stages; then the buffer is released
+  for (int i = 0; i < 3; ++i) {
+    cudaEvent_t end = ev[2 * nchunk + 1 + i];
+    if (cudaEventRecord(end, side[i]) != cudaSuccess || cudaStreamWaitEvent(s, end, 0) != cudaSuccess)
+      if (e == cudaSuccess) e = cudaErrorUnknown;
+  }
   if (cudaFreeAsync(buf, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  for (int i = 0; i < nev; ++i) cudaEventDestroy(ev[i]);
   g_last_launches = launches;
-  if (st != SAGE_OK) return st;
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 

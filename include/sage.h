@@ -273,10 +273,13 @@ SAGE_API sage_status sage_attn_decode(const void *q, const void *k, const void *
  * lives in host memory.  q/k/v/out are host pointers with the layouts of
  * sage_attn_fwd (pinned memory gives asynchronous copies; pageable memory
  * works but the copies then block the calling thread).  On `stream` the call
- * allocates device buffers (cudaMallocAsync), copies q, k, v to the device
- * (one cudaMemcpyAsync each), runs the forward pass, copies the output back
- * and frees the device buffers.  The host output is valid once `stream` has
- * been synchronized; the host buffers must stay alive until then.
+ * allocates device buffers (cudaMallocAsync) and frees them after the work;
+ * in between the (batch, kv head) groups are processed in up to 8 chunks
+ * through a three-stage pipeline on internal streams (copy in, compute, copy
+ * out; ordered after `stream`, and `stream` after them), so the copies of
+ * later chunks overlap the kernels of earlier ones.  The output is that of
+ * sage_attn_fwd, bit for bit.  The host output is valid once `stream` has been
+ * synchronized; the host buffers must stay alive until then.
  */
 SAGE_API sage_status sage_attn_fwd_host(const void *q_host, const void *k_host, const void *v_host,
                                void *out_host, int B, int H, int Hkv, int Lq, int Lk, int d,

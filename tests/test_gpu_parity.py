@@ -170,14 +170,20 @@ def test_deterministic():
     assert torch.equal(a, b)
 
 
-def test_host_buffer_entry_point_matches_device():
+@pytest.mark.parametrize("shape", [(1, 2, 2, 384, 384, 64, False),
+                                   (3, 8, 2, 300, 520, 128, True),    # 6 groups in 6 chunks
+                                   (4, 32, 8, 256, 256, 64, True)])   # 32 groups, 8 chunks
+def test_host_buffer_entry_point_matches_device(shape):
+    """The host-buffer call processes (batch, kv head) groups in chunks on two
+    side streams; its output must equal the device call's bit for bit."""
     torch = torch_mod()
-    q, k, v = inputs.make_custom(1, 2, 2, 384, 384, 64, seed=9)
+    B, H, Hkv, Lq, Lk, d, causal = shape
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=9 + B)
     hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
     hout = torch.empty(q.shape, dtype=torch.float16).pin_memory()
-    sage.sage_attn_fwd_host(hq, hk, hv, hout, False, 0.125)
+    sage.sage_attn_fwd_host(hq, hk, hv, hout, causal, 0.125)
     torch.cuda.current_stream().synchronize()
-    dev = sage.attention(to_dev(q), to_dev(k), to_dev(v), False, 0.125)
+    dev = sage.attention(to_dev(q), to_dev(k), to_dev(v), causal, 0.125)
     sage.sage_check_device_status()
     assert torch.equal(hout, dev.cpu())
 
