@@ -39,6 +39,7 @@ SYMBOLS = (
     "sage_quant_v_fp8",
     "sage_quant_v_fp8_workspace_size",
     "sage_attn_fwd_prequant_fp8pv",
+    "sage_attn_decode_prequant_varlen",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
@@ -117,6 +118,9 @@ def load_library():
         lib.sage_quant_v_fp8_workspace_size.restype = Z
         lib.sage_attn_fwd_prequant_fp8pv.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, P]
         lib.sage_attn_fwd_prequant_fp8pv.restype = I
+        lib.sage_attn_decode_prequant_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I,
+                                                         I, I, P, Z, P]
+        lib.sage_attn_decode_prequant_varlen.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -328,6 +332,19 @@ def sage_attn_decode_prequant(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_bl
                                                     int(q_block_rows), *_workspace(workspace),
                                                     _stream(stream)),
            "sage_attn_decode_prequant")
+
+
+def sage_attn_decode_prequant_varlen(q_i8, k_i8, q_scale, k_scale, v, out, seqlens_k, causal,
+                                     q_block_rows=128, workspace=None, stream=None):
+    """sage_attn_decode_prequant with one key count per batch entry
+    (seqlens_k: int32 CUDA tensor [B]) in a cache padded to Lk."""
+    import torch
+    _check_qbr(q_block_rows)
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
+    sl = _dev(seqlens_k, torch.int32, "seqlens_k", (q_i8.shape[0],))
+    _check(load_library().sage_attn_decode_prequant_varlen(
+        *args[:6], sl, *args[6:], 1 if causal else 0, int(q_block_rows), *_workspace(workspace),
+        _stream(stream)), "sage_attn_decode_prequant_varlen")
 
 
 def sage_attn_decode(q, k, v, out, causal, sm_scale, q_block_rows=128, stream=None):

@@ -13,7 +13,9 @@
 //     unnormalized partial output with its running max and sum; a second
 //     kernel merges the splits (skipped when nsplit = 1);
 //   * softmax warps whose 32 rows are all padding only keep the barrier
-//     protocol going, so a tile with few real rows costs little arithmetic.
+//     protocol going, so a tile with few real rows costs little arithmetic;
+//   * optionally each batch entry has its own number of keys (variable-length
+//     caches in one padded buffer): splits past an entry's length are empty.
 // Warp roles, tensor-memory layout, barriers and the bounded waits are those
 // of the forward kernel: warp 4 issues TMA loads, one thread of warp 5 the
 // tcgen05 MMAs, warps 0-3 own the rows.
@@ -78,8 +80,9 @@ __global__ void __launch_bounds__(192, 2)
 sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                    const float* __restrict__ k_scale, __half* __restrict__ out,
-                   float* __restrict__ o_part, float2* __restrict__ ml_part, int H, int Hkv, int G,
-                   int Lq, int Lk, int nsplit, int split_tiles, int qbr, int* status) {
+                   float* __restrict__ o_part, float2* __restrict__ ml_part,
+                   const int* __restrict__ seqlens, int H, int Hkv, int G, int Lq, int Lk,
+                   int nsplit, int split_tiles, int qbr, int* status) {
   using C = DecCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -91,9 +94,11 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int bhk = blockIdx.x / nsplit, sp = blockIdx.x - bhk * nsplit;
   const int b = bhk / Hkv, hkv = bhk - b * Hkv;
   const int rows = G * Lq;  // packed rows in use
-  const int nkb = (Lk + kDecKeys - 1) / kDecKeys;
+  const int nkb = (Lk + kDecKeys - 1) / kDecKeys;  // k_scale row length (the cache's)
+  // keys of this batch entry: all Lk, or its own length in a shared cache
+  const int Lb = seqlens ? min(max(__ldg(seqlens + b), 0), Lk) : Lk;
   const int t0 = sp * split_tiles;
-  const int nkt = max(0, min(nkb, t0 + split_tiles) - t0);
+  const int nkt = max(0, min((Lb + kDecKeys - 1) / kDecKeys, t0 + split_tiles) - t0);
 
   if (tid == 0) {
     for (int i = 0; i < C::NUM_BARS; ++i)
@@ -216,7 +221,7 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const int nqs = (Lq + qbr - 1) / qbr;
     const float sq = real ? __ldg(q_scale + (size_t)bh * nqs + i / qbr) : 0.f;
     const float* ks = k_scale + (size_t)bhk * nkb + t0;
-    const int diag = i + (Lk - Lq) + 1;  // keys [0, diag) visible to this row
+    const int diag = i + (Lb - Lq) + 1;  // keys [0, diag) visible to this row
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     float ck = nkt > 0 ? __ldg(ks) : 0.f;
@@ -234,7 +239,7 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         uint32_t s[64];
         tmem_ld64(s_tmem, s);
         const int key0 = (t0 + j) * kDecKeys;
-        int vis = real ? Lk - key0 : 0;
+        int vis = real ? Lb - key0 : 0;
         if (CAUSAL) vis = min(vis, diag - key0);
         const bool full = vis >= kDecKeys;
         int mx = INT_MIN;
@@ -452,7 +457,8 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const DecodePlan& p, cud
   const long long grid = (long long)a.B * a.Hkv * p.nsplit;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.out,
-                                                   a.o_part, a.ml_part, a.H, a.Hkv, G, a.Lq, a.Lk,
+                                                   a.o_part, a.ml_part, a.seqlens, a.H, a.Hkv, G,
+                                                   a.Lq, a.Lk,
                                                    p.nsplit, p.split_tiles, a.q_block_rows,
                                                    status);
   *launches += 1;

@@ -275,6 +275,17 @@ sage_status sage_attn_decode_prequant(const int8_t* q_i8, const int8_t* k_i8,
                                       void* out, int B, int H, int Hkv, int Lq, int Lk, int d,
                                       int causal, int q_block_rows, void* workspace,
                                       size_t workspace_bytes, void* stream) {
+  return sage_attn_decode_prequant_varlen(q_i8, k_i8, q_scale, k_scale, v, out, nullptr, B, H,
+                                          Hkv, Lq, Lk, d, causal, q_block_rows, workspace,
+                                          workspace_bytes, stream);
+}
+
+sage_status sage_attn_decode_prequant_varlen(const int8_t* q_i8, const int8_t* k_i8,
+                                             const float* q_scale, const float* k_scale,
+                                             const void* v, void* out, const int* seqlens_k,
+                                             int B, int H, int Hkv, int Lq, int Lk, int d,
+                                             int causal, int q_block_rows, void* workspace,
+                                             size_t workspace_bytes, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
@@ -297,7 +308,7 @@ sage_status sage_attn_decode_prequant(const int8_t* q_i8, const int8_t* k_i8,
   sage::DecodeArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                      static_cast<__half*>(out), need ? reinterpret_cast<float*>(ws) : nullptr,
                      need ? reinterpret_cast<float2*>(ws + p.o_bytes) : nullptr,
-                     B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows};
+                     B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows, seqlens_k};
   int launches = 0;
   cudaError_t e = sage::launch_decode(a, p, s, &launches);
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;

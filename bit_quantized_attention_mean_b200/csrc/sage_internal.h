@@ -64,6 +64,7 @@ struct DecodeArgs {
   int B, H, Hkv, Lq, Lk, d;
   bool causal;
   int q_block_rows;
+  const int* seqlens = nullptr;  // [B] keys per batch entry (<= Lk), or null: all Lk
 };
 
 struct DecodePlan {

@@ -256,6 +256,22 @@ SAGE_API sage_status sage_attn_decode_prequant(const int8_t *q_i8, const int8_t 
                                    int causal, int q_block_rows,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * sage_attn_decode_prequant_varlen -- sage_attn_decode_prequant for a batch
+ * whose entries hold different numbers of keys in one padded cache: entry b
+ * uses keys [0, seqlens_k[b]) of its [Lk, d] rows (seqlens_k: device int32
+ * [B], values clamped to [0, Lk]; key blocks and their k_scale entries past an
+ * entry's length are not read).  Causal masking is bottom-right aligned to
+ * seqlens_k[b]; an entry with no keys outputs zeros.  K of each entry must
+ * have been smoothed and quantized over its own keys (its own mean).
+ */
+SAGE_API sage_status sage_attn_decode_prequant_varlen(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out, const int *seqlens_k,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of scratch sage_attn_decode_prequant needs (0 for unsupported shapes). */
 SAGE_API size_t sage_attn_decode_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
 

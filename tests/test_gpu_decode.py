@@ -106,3 +106,38 @@ def test_decode_full_size_sampled_rows():
     sim = oracle.attn_quant_sim(*qk[:4], v, True, rows=rows, q_block_rows=1)
     ref = oracle.attn_fp64(q, k, v, True, sm, rows=rows)
     assert_close(out, sim, ref, "decode B8 H32 Hkv8 Lq1 Lk32768 d128")
+
+
+@pytest.mark.parametrize("Lq,causal", [(1, True), (4, True), (3, False)])
+def test_decode_varlen_against_oracle(Lq, causal):
+    """Entries with 4096, 777, 65, 1 and 0 keys in one padded 4096-key cache:
+    each entry's K is smoothed and quantized over its own keys (the oracle,
+    per entry), and the kernel must read only those keys."""
+    torch = torch_mod()
+    B, H, Hkv, Lk, d = 5, 8, 2, 4096, 128
+    lens = [4096, 777, 65, 1, 0]
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=94 + Lq, k_offset_sigma=2.0)
+    sm = float(np.float32(1 / math.sqrt(d)))
+    qbr = 1
+    nkb = Lk // 64
+    k_i8 = np.zeros((B, Hkv, Lk, d), np.int8)
+    k_scale = np.zeros((B, Hkv, nkb), np.float32)
+    q_i8 = np.zeros((B, H, Lq, d), np.int8)
+    q_scale = np.zeros((B, H, Lq), np.float32)
+    want = np.zeros((B, H, Lq, d))
+    for b, L in enumerate(lens):
+        Lb = max(L, 1)   # the oracle needs one key to quantize; length 0 reads none
+        qk = oracle.quant_qk(q[b:b + 1], k[b:b + 1, :, :Lb], sm, q_block_rows=qbr)
+        q_i8[b], q_scale[b] = qk[0][0], qk[2][0]
+        k_i8[b, :, :Lb], k_scale[b, :, :-(-Lb // 64)] = qk[1][0], qk[3][0]
+        if L > 0:
+            want[b] = oracle.attn_quant_sim(qk[0], qk[1], qk[2], qk[3], v[b:b + 1, :, :L],
+                                            causal, q_block_rows=qbr)[0]
+    out = torch.empty((B, H, Lq, d), dtype=torch.float16, device="cuda")
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    sage.sage_attn_decode_prequant_varlen(to_dev(q_i8), to_dev(k_i8), to_dev(q_scale),
+                                          to_dev(k_scale), to_dev(v), out, sl, causal, qbr)
+    sage.sage_check_device_status()
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(got[4] == 0)
+    assert_close(got[:4], want[:4], None, f"varlen Lq={Lq} causal={causal}")
