@@ -50,6 +50,7 @@ from ._lib import (  # noqa: F401
     sage_attn_decode_prequant,
     sage_attn_decode_workspace_size,
     sage_attn_decode_prequant_varlen,
+    sage_attn_decode_prequant_paged,
     sage_quant_v_fp8,
     sage_quant_v_fp8_workspace_size,
     sage_attn_fwd_prequant_fp8pv,

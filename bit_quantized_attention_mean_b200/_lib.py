@@ -40,6 +40,7 @@ SYMBOLS = (
     "sage_quant_v_fp8_workspace_size",
     "sage_attn_fwd_prequant_fp8pv",
     "sage_attn_decode_prequant_varlen",
+    "sage_attn_decode_prequant_paged",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
@@ -121,6 +122,9 @@ def load_library():
         lib.sage_attn_decode_prequant_varlen.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I,
                                                          I, I, P, Z, P]
         lib.sage_attn_decode_prequant_varlen.restype = I
+        lib.sage_attn_decode_prequant_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
+                                                        I, I, I, P, Z, P]
+        lib.sage_attn_decode_prequant_paged.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -345,6 +349,30 @@ def sage_attn_decode_prequant_varlen(q_i8, k_i8, q_scale, k_scale, v, out, seqle
     _check(load_library().sage_attn_decode_prequant_varlen(
         *args[:6], sl, *args[6:], 1 if causal else 0, int(q_block_rows), *_workspace(workspace),
         _stream(stream)), "sage_attn_decode_prequant_varlen")
+
+
+def sage_attn_decode_prequant_paged(q_i8, q_scale, k_pages, k_scale_pages, v_pages, block_table,
+                                    seqlens_k, out, causal, q_block_rows=128, workspace=None,
+                                    stream=None):
+    """Decoding on a paged cache: k_pages int8 / v_pages fp16 [num_pages, Hkv,
+    64, d], k_scale_pages [num_pages, Hkv], block_table int32 [B, max_blocks],
+    seqlens_k int32 [B] (all CUDA tensors)."""
+    import torch
+    _check_qbr(q_block_rows)
+    B, H, Lq, d = q_i8.shape
+    num_pages, Hkv = k_pages.shape[0], k_pages.shape[1]
+    max_blocks = block_table.shape[1]
+    nqb = -(-Lq // q_block_rows)
+    _check(load_library().sage_attn_decode_prequant_paged(
+        _dev(q_i8, torch.int8, "q_i8"), _dev(q_scale, torch.float32, "q_scale", (B, H, nqb)),
+        _dev(k_pages, torch.int8, "k_pages", (num_pages, Hkv, 64, d)),
+        _dev(k_scale_pages, torch.float32, "k_scale_pages", (num_pages, Hkv)),
+        _dev(v_pages, torch.float16, "v_pages", (num_pages, Hkv, 64, d)),
+        _dev(block_table, torch.int32, "block_table", (B, max_blocks)),
+        _dev(seqlens_k, torch.int32, "seqlens_k", (B,)),
+        _dev(out, torch.float16, "out", q_i8.shape), B, H, Hkv, Lq, num_pages, max_blocks, d,
+        1 if causal else 0, int(q_block_rows), *_workspace(workspace), _stream(stream)),
+        "sage_attn_decode_prequant_paged")
 
 
 def sage_attn_decode(q, k, v, out, causal, sm_scale, q_block_rows=128, stream=None):

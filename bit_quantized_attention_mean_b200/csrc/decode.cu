@@ -15,7 +15,9 @@
 //   * softmax warps whose 32 rows are all padding only keep the barrier
 //     protocol going, so a tile with few real rows costs little arithmetic;
 //   * optionally each batch entry has its own number of keys (variable-length
-//     caches in one padded buffer): splits past an entry's length are empty.
+//     caches in one padded buffer): splits past an entry's length are empty;
+//   * optionally the cache is paged: 64-key pages (one K quantization block
+//     each) of all kv heads, found through a per-entry block table.
 // Warp roles, tensor-memory layout, barriers and the bounded waits are those
 // of the forward kernel: warp 4 issues TMA loads, one thread of warp 5 the
 // tcgen05 MMAs, warps 0-3 own the rows.
@@ -81,7 +83,8 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                    const float* __restrict__ k_scale, __half* __restrict__ out,
                    float* __restrict__ o_part, float2* __restrict__ ml_part,
-                   const int* __restrict__ seqlens, int H, int Hkv, int G, int Lq, int Lk,
+                   const int* __restrict__ seqlens, const int* __restrict__ block_table,
+                   int max_blocks, int num_pages, int H, int Hkv, int G, int Lq, int Lk,
                    int nsplit, int split_tiles, int qbr, int* status) {
   using C = DecCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -99,6 +102,12 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int Lb = seqlens ? min(max(__ldg(seqlens + b), 0), Lk) : Lk;
   const int t0 = sp * split_tiles;
   const int nkt = max(0, min((Lb + kDecKeys - 1) / kDecKeys, t0 + split_tiles) - t0);
+  // Paged caches: key tile t of entry b is page block_table[b][t] (64 keys of
+  // every kv head); its K/V rows are at TMA coordinate z = page * Hkv + hkv
+  // and its k_scale at [page][hkv].  Pages outside [0, num_pages) are clamped.
+  auto page_of = [&](int t) {
+    return min(max(__ldg(block_table + (size_t)b * max_blocks + t), 0), num_pages - 1);
+  };
 
   if (tid == 0) {
     for (int i = 0; i < C::NUM_BARS; ++i)
@@ -140,13 +149,18 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
             !mbar_wait(&bars[C::B_KV_EMPTY + s], ((j / C::STAGES) - 1) & 1, abort_flag, status, 31))
           break;
         mbar_arrive_expect_tx(&bars[C::B_K_FULL + s], C::K_BYTES);
-        tma_load_3d_hint(smem + C::OFF_K + s * C::K_BYTES, &tm_k, &bars[C::B_K_FULL + s], 0,
-                         (t0 + j) * kDecKeys, bhk, stream);
+        int ky = (t0 + j) * kDecKeys, kz = bhk;
+        if (block_table) {
+          ky = 0;
+          kz = page_of(t0 + j) * Hkv + hkv;
+        }
+        tma_load_3d_hint(smem + C::OFF_K + s * C::K_BYTES, &tm_k, &bars[C::B_K_FULL + s], 0, ky,
+                         kz, stream);
         mbar_arrive_expect_tx(&bars[C::B_V_FULL + s], C::V_BYTES);
 #pragma unroll
         for (int cc = 0; cc < D / 64; ++cc)
           tma_load_3d_hint(smem + C::OFF_V + s * C::V_BYTES + cc * (kDecKeys * 128), &tm_v,
-                           &bars[C::B_V_FULL + s], cc * 64, (t0 + j) * kDecKeys, bhk, stream);
+                           &bars[C::B_V_FULL + s], cc * 64, ky, kz, stream);
         issued = j + 1;
       }
       mbar_wait_drain(&bars[C::B_Q_FULL], 0);
@@ -220,15 +234,18 @@ sage_decode_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const int nqs = (Lq + qbr - 1) / qbr;
     const float sq = real ? __ldg(q_scale + (size_t)bh * nqs + i / qbr) : 0.f;
-    const float* ks = k_scale + (size_t)bhk * nkb + t0;
+    auto kscale = [&](int t) {
+      return __ldg(block_table ? k_scale + (size_t)page_of(t) * Hkv + hkv
+                               : k_scale + (size_t)bhk * nkb + t);
+    };
     const int diag = i + (Lb - Lq) + 1;  // keys [0, diag) visible to this row
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    float ck = nkt > 0 ? __ldg(ks) : 0.f;
+    float ck = nkt > 0 ? kscale(t0) : 0.f;
     for (int j = 0; j < nkt; ++j) {
       const int bb = j & 1;
       const float c = __fmul_rn(sq, ck);
-      if (j + 1 < nkt) ck = __ldg(ks + j + 1);
+      if (j + 1 < nkt) ck = kscale(t0 + j + 1);
       if (!dec_warp_wait(&bars[C::B_S_FULL + bb], (j >> 1) & 1, abort_flag, status, 36)) {
         ok = false;
         break;
@@ -444,7 +461,9 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const DecodePlan& p, cud
   CUtensorMap tq, tk, tv;
   const uint64_t qd[4] = {(uint64_t)D, (uint64_t)a.Lq, (uint64_t)G, (uint64_t)a.B * a.Hkv};
   const uint32_t qb[4] = {(uint32_t)D, (uint32_t)a.Lq, (uint32_t)G, 1u};
-  const uint64_t kd[3] = {(uint64_t)D, (uint64_t)a.Lk, (uint64_t)a.B * a.Hkv};
+  // contiguous cache [B*Hkv, Lk, d]; paged cache [num_pages*Hkv, 64, d]
+  const uint64_t kd[3] = {(uint64_t)D, a.block_table ? (uint64_t)kDecKeys : (uint64_t)a.Lk,
+                          a.block_table ? (uint64_t)a.num_pages * a.Hkv : (uint64_t)a.B * a.Hkv};
   const uint32_t kb[3] = {(uint32_t)D, (uint32_t)kDecKeys, 1u};
   const uint32_t vb[3] = {64u, (uint32_t)kDecKeys, 1u};
   if (!dec_make_map(&tq, a.q_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, 4, qd, qb, qk_sw) ||
@@ -457,7 +476,8 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, const DecodePlan& p, cud
   const long long grid = (long long)a.B * a.Hkv * p.nsplit;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.out,
-                                                   a.o_part, a.ml_part, a.seqlens, a.H, a.Hkv, G,
+                                                   a.o_part, a.ml_part, a.seqlens, a.block_table,
+                                                   a.max_blocks, a.num_pages, a.H, a.Hkv, G,
                                                    a.Lq, a.Lk,
                                                    p.nsplit, p.split_tiles, a.q_block_rows,
                                                    status);

@@ -316,6 +316,52 @@ sage_status sage_attn_decode_prequant_varlen(const int8_t* q_i8, const int8_t* k
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
+sage_status sage_attn_decode_prequant_paged(const int8_t* q_i8, const float* q_scale,
+                                            const int8_t* k_pages, const float* k_scale_pages,
+                                            const void* v_pages, const int* block_table,
+                                            const int* seqlens_k, void* out, int B, int H,
+                                            int Hkv, int Lq, int num_pages, int max_blocks, int d,
+                                            int causal, int q_block_rows, void* workspace,
+                                            size_t workspace_bytes, void* stream) {
+  g_last_launches = 0;
+  if (num_pages < 1 || max_blocks < 1 || (long long)max_blocks * 64 > 0x7fffffffLL)
+    return SAGE_ERR_INVALID_ARG;
+  const int Lk = max_blocks * 64;
+  sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
+  if (st != SAGE_OK) return st;
+  if ((long long)num_pages * Hkv * 64 * d > (1LL << 40)) return SAGE_ERR_INVALID_ARG;
+  if ((long long)(H / Hkv) * Lq > 128) return SAGE_ERR_UNSUPPORTED;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
+  if (!q_i8 || !q_scale || !k_pages || !k_scale_pages || !v_pages || !block_table || !seqlens_k ||
+      !out)
+    return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q_i8) || !aligned16(k_pages) || !aligned16(v_pages) || !aligned16(out) ||
+      !aligned16(q_scale) || !aligned16(k_scale_pages))
+    return SAGE_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  const sage::DecodePlan p = sage::decode_plan(B, H, Hkv, Lq, Lk, d);
+  const size_t need = p.o_bytes + p.ml_bytes;
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  char* ws = static_cast<char*>(workspace);
+  const bool own = !ws && need > 0;
+  if (own && cudaMallocAsync(reinterpret_cast<void**>(&ws), need, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  sage::DecodeArgs a{q_i8, k_pages, q_scale, k_scale_pages, static_cast<const __half*>(v_pages),
+                     static_cast<__half*>(out), need ? reinterpret_cast<float*>(ws) : nullptr,
+                     need ? reinterpret_cast<float2*>(ws + p.o_bytes) : nullptr,
+                     B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows, seqlens_k};
+  a.block_table = block_table;
+  a.max_blocks = max_blocks;
+  a.num_pages = num_pages;
+  int launches = 0;
+  cudaError_t e = sage::launch_decode(a, p, s, &launches);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
 sage_status sage_attn_decode(const void* q, const void* k, const void* v, void* out, int B, int H,
                              int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
                              int q_block_rows, void* stream) {

@@ -65,6 +65,10 @@ struct DecodeArgs {
   bool causal;
   int q_block_rows;
   const int* seqlens = nullptr;  // [B] keys per batch entry (<= Lk), or null: all Lk
+  // paged cache: k_i8/v are [num_pages, Hkv, 64, d], k_scale [num_pages, Hkv],
+  // block_table [B, max_blocks] page indices, Lk = 64 * max_blocks
+  const int* block_table = nullptr;
+  int max_blocks = 0, num_pages = 0;
 };
 
 struct DecodePlan {

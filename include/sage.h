@@ -272,6 +272,27 @@ SAGE_API sage_status sage_attn_decode_prequant_varlen(const int8_t *q_i8, const 
                                    int causal, int q_block_rows,
                                    void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * sage_attn_decode_prequant_paged -- the decoding layout on a paged cache.
+ * A page holds 64 consecutive keys (one K quantization block) of every kv
+ * head: k_pages int8 [num_pages, Hkv, 64, d], v_pages fp16 [num_pages, Hkv,
+ * 64, d], k_scale_pages fp32 [num_pages, Hkv] (the scale of that block).
+ * block_table int32 [B, max_blocks] (device) lists entry b's pages in key
+ * order; seqlens_k int32 [B] (device) its key counts (clamped to
+ * [0, 64 * max_blocks]); page indices outside [0, num_pages) are clamped.
+ * q_i8, q_scale, out, causal, q_block_rows, workspace: as
+ * sage_attn_decode_prequant with Lk = 64 * max_blocks (also for
+ * sage_attn_decode_workspace_size).  K of each entry must have been smoothed
+ * and quantized over its own keys.
+ */
+SAGE_API sage_status sage_attn_decode_prequant_paged(const int8_t *q_i8, const float *q_scale,
+                                   const int8_t *k_pages, const float *k_scale_pages,
+                                   const void *v_pages, const int *block_table,
+                                   const int *seqlens_k, void *out,
+                                   int B, int H, int Hkv, int Lq, int num_pages, int max_blocks,
+                                   int d, int causal, int q_block_rows,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of scratch sage_attn_decode_prequant needs (0 for unsupported shapes). */
 SAGE_API size_t sage_attn_decode_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
 

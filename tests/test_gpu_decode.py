@@ -141,3 +141,47 @@ def test_decode_varlen_against_oracle(Lq, causal):
     got = out.cpu().numpy().astype(np.float64)
     assert np.all(got[4] == 0)
     assert_close(got[:4], want[:4], None, f"varlen Lq={Lq} causal={causal}")
+
+
+def test_decode_paged_equals_contiguous_varlen():
+    """The same per-entry caches laid out as shuffled 64-key pages through a
+    block table must give the contiguous variable-length result bit for bit
+    (same arithmetic, different addressing)."""
+    torch = torch_mod()
+    B, H, Hkv, Lq, Lk, d = 4, 16, 4, 2, 2048, 128
+    lens = [2048, 1000, 64, 3]
+    q, k, v = inputs.make_custom(B, H, Hkv, Lq, Lk, d, seed=97, k_offset_sigma=2.0)
+    sm, qbr = 0.088, 1
+    nkb = Lk // 64
+    k_i8 = np.zeros((B, Hkv, Lk, d), np.int8)
+    k_scale = np.zeros((B, Hkv, nkb), np.float32)
+    q_i8 = np.zeros((B, H, Lq, d), np.int8)
+    q_scale = np.zeros((B, H, Lq), np.float32)
+    for b, L in enumerate(lens):
+        qk = oracle.quant_qk(q[b:b + 1], k[b:b + 1, :, :L], sm, q_block_rows=qbr)
+        q_i8[b], q_scale[b] = qk[0][0], qk[2][0]
+        k_i8[b, :, :L], k_scale[b, :, :-(-L // 64)] = qk[1][0], qk[3][0]
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    dq, dqs, dv = to_dev(q_i8), to_dev(q_scale), to_dev(v)
+    ref = torch.empty((B, H, Lq, d), dtype=torch.float16, device="cuda")
+    sage.sage_attn_decode_prequant_varlen(dq, to_dev(k_i8), dqs, to_dev(k_scale), dv, ref, sl,
+                                          True, qbr)
+    # pages: every used 64-key block of every entry gets a distinct page, shuffled
+    rng = np.random.default_rng(5)
+    used = [(b, t) for b, L in enumerate(lens) for t in range(-(-L // 64))]
+    npages = len(used) + 7                      # a few pages nobody uses
+    order = rng.permutation(npages)[:len(used)]
+    k_pages = np.zeros((npages, Hkv, 64, d), np.int8)
+    v_pages = np.zeros((npages, Hkv, 64, d), np.float16)
+    ks_pages = np.zeros((npages, Hkv), np.float32)
+    table = np.full((B, nkb), npages - 1, np.int32)  # unused slots point anywhere valid
+    for (b, t), pg in zip(used, order):
+        k_pages[pg] = k_i8[b, :, t * 64:(t + 1) * 64]
+        v_pages[pg] = v[b, :, t * 64:(t + 1) * 64]
+        ks_pages[pg] = k_scale[b, :, t]
+        table[b, t] = pg
+    out = torch.empty_like(ref)
+    sage.sage_attn_decode_prequant_paged(dq, dqs, to_dev(k_pages), to_dev(ks_pages),
+                                         to_dev(v_pages), to_dev(table), sl, out, True, qbr)
+    sage.sage_check_device_status()
+    assert torch.equal(out, ref)
