@@ -263,3 +263,25 @@ def test_workload(idx):
     ref = oracle.attn_fp64(q, k, v, w.causal, sm, rows=rows).reshape(-1, w.d)
     got = out if rows is None else out[rows]
     assert_close(got, sim, ref, w.name)
+
+
+def test_degenerate_blocks_zero_q_and_constant_k():
+    """An all-zero 128-row Q block (scale 0) and a head whose K rows are all
+    equal (smoothed K is 0, every K scale 0) quantize to zero codes with zero
+    scales and give uniform attention over the visible keys."""
+    torch = torch_mod()
+    B, H, L, d = 1, 2, 300, 128
+    q, k, v = inputs.make_custom(B, H, H, L, L, d, seed=71)
+    q[0, 0, 128:256] = 0                            # zero Q block of head 0
+    k[0, 1] = k[0, 1, :1]                           # constant K rows in head 1
+    sm = 1 / math.sqrt(d)
+    want = oracle.quant_qk(q, k, sm)
+    got = gpu_quant(q, k, sm)
+    assert_quant_bitexact(got, want, "degenerate blocks")
+    assert got[2][0, 0, 1] == 0 and np.all(got[0][0, 0, 128:256] == 0)
+    assert np.all(got[3][0, 1] == 0) and np.all(got[1][0, 1] == 0)
+    out = gpu_attention(q, k, v, True, sm).astype(np.float64)
+    vv = v.astype(np.float64)
+    uniform = np.cumsum(vv, axis=2) / np.arange(1, L + 1)[None, None, :, None]
+    assert np.abs(out[0, 0, 128:256] - uniform[0, 0, 128:256]).max() <= 2e-3
+    assert np.abs(out[0, 1] - uniform[0, 1]).max() <= 2e-3
