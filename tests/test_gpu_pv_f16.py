@@ -98,7 +98,7 @@ def test_unknown_flags_are_rejected():
     q = torch.zeros((1, 1, 128, 64), dtype=torch.float16, device="cuda")
     out = torch.empty_like(q)
     P = ctypes.c_void_p
-    for bad in (2, 4, 0x80000000, 3):
+    for bad in (4, 8, 0x80000000, 3):   # 3 = both P V variants at once
         st = lib.sage_attn_fwd_ex(P(q.data_ptr()), P(q.data_ptr()), P(q.data_ptr()),
                                   P(out.data_ptr()), 1, 1, 1, 128, 128, 64, 0, 0.125, 128, bad,
                                   P(torch.cuda.current_stream().cuda_stream))
