@@ -41,6 +41,9 @@ SYMBOLS = (
     "sage_attn_fwd_prequant_fp8pv",
     "sage_attn_decode_prequant_varlen",
     "sage_attn_decode_prequant_paged",
+    "sage_quant_qk_varlen",
+    "sage_attn_fwd_prequant_varlen",
+    "sage_attn_fwd_varlen",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
@@ -125,6 +128,14 @@ def load_library():
         lib.sage_attn_decode_prequant_paged.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
                                                         I, I, I, P, Z, P]
         lib.sage_attn_decode_prequant_paged.restype = I
+        lib.sage_quant_qk_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I,
+                                             P, Z, P]
+        lib.sage_quant_qk_varlen.restype = I
+        lib.sage_attn_fwd_prequant_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
+                                                      I, I, U, P]
+        lib.sage_attn_fwd_prequant_varlen.restype = I
+        lib.sage_attn_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P]
+        lib.sage_attn_fwd_varlen.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -320,6 +331,63 @@ def sage_attn_fwd_prequant_ex(q_i8, k_i8, q_scale, k_scale, v, out, causal, q_bl
     _check(load_library().sage_attn_fwd_prequant_ex(*args, 1 if causal else 0,
                                                     int(q_block_rows), flags, _stream(stream)),
            "sage_attn_fwd_prequant_ex")
+
+
+def _seqlens(t, name, B):
+    """Device pointer of an optional int32 [B] length tensor (None -> NULL)."""
+    import torch
+    if t is None:
+        return ctypes.c_void_p(0)
+    return _dev(t, torch.int32, name, (B,))
+
+
+def sage_quant_qk_varlen(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, seqlens_q, seqlens_k,
+                         sm_scale, q_block_rows=128, workspace=None, stream=None):
+    """sage_quant_qk_qblock on a padded batch: entry b quantizes its first
+    seqlens_q[b] Q rows and smooths/quantizes its first seqlens_k[b] keys
+    (int32 CUDA tensors [B], or None for all rows / all keys)."""
+    _check_qbr(q_block_rows)
+    args = _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, q_block_rows)
+    B = q.shape[0]
+    _check(load_library().sage_quant_qk_varlen(
+        *args[:7], _seqlens(seqlens_q, "seqlens_q", B), _seqlens(seqlens_k, "seqlens_k", B),
+        *args[7:], float(sm_scale), int(q_block_rows), *_workspace(workspace), _stream(stream)),
+        "sage_quant_qk_varlen")
+
+
+def sage_attn_fwd_prequant_varlen(q_i8, k_i8, q_scale, k_scale, v, out, seqlens_q, seqlens_k,
+                                  causal, q_block_rows=128, pv_accum="f32", stream=None):
+    """sage_attn_fwd_prequant_ex on a padded batch (lengths as
+    sage_quant_qk_varlen); output rows past seqlens_q[b] are written as zeros."""
+    _check_qbr(q_block_rows)
+    flags = _flags(pv_accum)
+    if flags == SAGE_PV_FP8:
+        raise ValueError("sage_attn_fwd_prequant_varlen takes fp16 V (pv_accum 'f32' or 'f16')")
+    args = _prequant_args(q_i8, k_i8, q_scale, k_scale, v, out, q_block_rows)
+    B = q_i8.shape[0]
+    _check(load_library().sage_attn_fwd_prequant_varlen(
+        *args[:6], _seqlens(seqlens_q, "seqlens_q", B), _seqlens(seqlens_k, "seqlens_k", B),
+        *args[6:], 1 if causal else 0, int(q_block_rows), flags, _stream(stream)),
+        "sage_attn_fwd_prequant_varlen")
+
+
+def sage_attn_fwd_varlen(q, k, v, out, seqlens_q, seqlens_k, causal, sm_scale, q_block_rows=128,
+                         pv_accum="f32", stream=None):
+    """The whole forward pass on a padded batch: entry b attends with its
+    first seqlens_q[b] rows over its first seqlens_k[b] keys, exactly as the
+    same call on that entry alone; padding output rows are zeros and the V
+    padding inside an entry's last 64-key tile must be finite."""
+    import torch
+    _check_qbr(q_block_rows)
+    flags = _flags(pv_accum)
+    lib = load_library()
+    B, H, Hkv, Lq, Lk, d = _dims(q, k)
+    _check(lib.sage_attn_fwd_varlen(
+        _dev(q, torch.float16, "q"), _dev(k, torch.float16, "k"),
+        _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
+        _seqlens(seqlens_q, "seqlens_q", B), _seqlens(seqlens_k, "seqlens_k", B),
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows), flags,
+        _stream(stream)), "sage_attn_fwd_varlen")
 
 
 def sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
@@ -521,6 +589,19 @@ def quant_qk(q, k, sm_scale, q_block_rows=128, stream=None):
         sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
                              q_block_rows, stream=stream)
     return q_i8, k_i8, q_scale, k_scale, k_mean
+
+
+def attention_varlen(q, k, v, seqlens_q=None, seqlens_k=None, causal=False, sm_scale=None,
+                     q_block_rows=128, pv_accum="f32", stream=None):
+    """Allocate the output and run sage_attn_fwd_varlen on a padded batch;
+    returns the fp16 output (zeros past each entry's seqlens_q)."""
+    import torch
+    if sm_scale is None:
+        sm_scale = q.shape[-1] ** -0.5
+    out = torch.empty_like(q)
+    sage_attn_fwd_varlen(q, k, v, out, seqlens_q, seqlens_k, causal, sm_scale, q_block_rows,
+                         pv_accum, stream=stream)
+    return out
 
 
 def attention(q, k, v, causal=False, sm_scale=None, q_block_rows=128, pv_accum="f32",

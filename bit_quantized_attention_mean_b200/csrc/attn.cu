@@ -124,7 +124,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const __grid_constant__ CUtensorMap tm_v, const float* __restrict__ q_scale,
                      const float* __restrict__ k_scale, const float* __restrict__ v_scale,
                      __half* __restrict__ out, int H, int Hkv, int Lq, int Lk, int nqt,
-                     int global_lpt, int qbr) {
+                     int global_lpt, int qbr, const int* __restrict__ seqlens_q,
+                     const int* __restrict__ seqlens_k) {
   constexpr bool F16ACC = PV == kPvF16Acc;
   constexpr bool FP8V = PV == kPvFp8;
   using C = AttnCfg<D, FP8V>;
@@ -152,12 +153,16 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int h = bh % H, b = bh / H;
   const int bhk = b * Hkv + h / (H / Hkv);
   const int q0 = qt * BQ;
-  const int nkb = (Lk + BK - 1) / BK;
-  int nkt = nkb;
-  if (CAUSAL) {
-    const int last_row = min(q0 + BQ, Lq) - 1;
-    const int vis = last_row + (Lk - Lq) + 1;  // keys [0, vis) visible to the tile's last row
-    nkt = vis <= 0 ? 0 : min(nkb, (vis + BK - 1) / BK);
+  const int nkb = (Lk + BK - 1) / BK;  // k_scale row length
+  // rows and keys of this batch entry: all of them, or its own counts in a
+  // padded batch (rows past Lqb are written as zeros)
+  const int Lqb = seqlens_q ? min(max(__ldg(seqlens_q + b), 0), Lq) : Lq;
+  const int Lkb = seqlens_k ? min(max(__ldg(seqlens_k + b), 0), Lk) : Lk;
+  int nkt = q0 < Lqb ? (Lkb + BK - 1) / BK : 0;
+  if (CAUSAL && nkt > 0) {
+    const int last_row = min(q0 + BQ, Lqb) - 1;
+    const int vis = last_row + (Lkb - Lqb) + 1;  // keys [0, vis) visible to the tile's last row
+    nkt = vis <= 0 ? 0 : min(nkt, (vis + BK - 1) / BK);
   }
 
   if (tid == 0) {
@@ -298,9 +303,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     // this row's Q scale (blocks of qbr rows; padding rows reuse the last)
     const int nqs = (Lq + qbr - 1) / qbr;
-    const float sq = __ldg(q_scale + (size_t)bh * nqs + min(qrow, Lq - 1) / qbr);
+    const bool real = qrow < Lqb;
+    const float sq = real ? __ldg(q_scale + (size_t)bh * nqs + qrow / qbr) : 0.f;
     const float* ks = k_scale + (size_t)bhk * nkb;
-    const int diag = qrow + (Lk - Lq) + 1;  // keys [0, diag) visible to this row
+    const int diag = real ? qrow + (Lkb - Lqb) + 1 : 0;  // keys [0, diag) visible to this row
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     float ck = nkt > 0 ? __ldg(ks) : 0.f;
@@ -317,7 +323,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       uint32_t s[64];
       tmem_ld64(s_tmem, s);
 
-      int vis = Lk - j * BK;
+      int vis = real ? Lkb - j * BK : 0;
       if (CAUSAL) vis = min(vis, diag - j * BK);
       const bool full = vis >= BK;
       int mx = INT_MIN;
@@ -498,7 +504,7 @@ static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launch
   kern<<<(unsigned)grid, 192, C::SMEM_BYTES, st>>>(tq, tk, tv, a.q_scale, a.k_scale, a.v_scale,
                                                    a.out, a.H, a.Hkv, a.Lq, a.Lk, nqt,
                                                    kv_bytes <= kGlobalOrderKVBytes ? 1 : 0,
-                                                   a.q_block_rows);
+                                                   a.q_block_rows, a.seqlens_q, a.seqlens_k);
   *launches += 1;
   return cudaGetLastError();
 }

@@ -228,7 +228,9 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
                 int8_t* __restrict__ q_i8, int8_t* __restrict__ k_i8,
                 float* __restrict__ q_scale, float* __restrict__ k_scale,
                 float* __restrict__ k_mean, int BHkv, int Lq, int Lk, int nqb, int nkb,
-                int kb_per_cta, int n_k_ctas, int n_q_blocks, float c) {
+                int kb_per_cta, int n_k_ctas, int n_q_blocks, float c,
+                const int* __restrict__ seqlens_q, const int* __restrict__ seqlens_k, int H,
+                int Hkv) {
   constexpr int TPR = D / 8;
   constexpr int RPP = kQuantThreads / TPR;  // rows per pass of the column sums
   __shared__ float red[32];
@@ -243,10 +245,13 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
     if (blk >= n_q_blocks) return;  // padding CTA of the last cluster
     const int bh = blk / nqb, qb = blk - bh * nqb;
     const int r0 = qb * SAGE_Q_BLOCK_ROWS;
+    // rows of this head: all Lq, or the entry's own count in a padded batch
+    const int Lqb = seqlens_q ? min(max(__ldg(seqlens_q + bh / H), 0), Lq) : Lq;
+    if (r0 >= Lqb) return;  // padding rows only
     const size_t off = ((size_t)bh * Lq + r0) * D;
     const int nqs = (Lq + QBR - 1) / QBR;  // scales per head
     quant_q_tile<D, QBR>(q + off, q_i8 + off, q_scale + (size_t)bh * nqs + r0 / QBR,
-                         min(SAGE_Q_BLOCK_ROWS, Lq - r0), c, red);
+                         min(SAGE_Q_BLOCK_ROWS, Lqb - r0), c, red);
     return;
   }
 
@@ -255,8 +260,11 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   const int ncl = (int)cluster.num_blocks();
   const int rank = (int)cluster.block_rank();
   const int bhk = blockIdx.x / ncl;
-  const int kb0 = min(nkb, rank * kb_per_cta), kb1 = min(nkb, kb0 + kb_per_cta);
-  const int t0 = kb0 * SAGE_K_BLOCK_ROWS, t1 = min(Lk, kb1 * SAGE_K_BLOCK_ROWS);
+  // keys of this head: all Lk, or the entry's own count in a padded batch
+  const int Lkb = seqlens_k ? min(max(__ldg(seqlens_k + bhk / Hkv), 0), Lk) : Lk;
+  const int nkb_b = (Lkb + SAGE_K_BLOCK_ROWS - 1) / SAGE_K_BLOCK_ROWS;
+  const int kb0 = min(nkb_b, rank * kb_per_cta), kb1 = min(nkb_b, kb0 + kb_per_cta);
+  const int t0 = kb0 * SAGE_K_BLOCK_ROWS, t1 = min(Lkb, kb1 * SAGE_K_BLOCK_ROWS);
   const __half* kh = k + (size_t)bhk * Lk * D;
 
   // pass 1: exact column sums of rows [t0, t1)
@@ -288,7 +296,7 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   for (int ch = tid; ch < D; ch += kQuantThreads) {
     long long s = 0;
     for (int r = 0; r < ncl; ++r) s += *cluster.map_shared_rank(&part[ch], r);
-    const double mu = __ddiv_rn(__dmul_rn(__ll2double_rn(s), 0x1p-24), (double)Lk);
+    const double mu = Lkb > 0 ? __ddiv_rn(__dmul_rn(__ll2double_rn(s), 0x1p-24), (double)Lkb) : 0.0;
     mean[ch] = __double2float_rn(mu);
     if (rank == 0) k_mean[(size_t)bhk * D + ch] = mean[ch];
   }
@@ -300,7 +308,7 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   for (int e = 0; e < 8; ++e) m8[e] = mean[(tid % TPR) * 8 + e];
   for (int kb = kb0; kb < kb1; kb += 2)
     quant_k_blocks<D, 2>(k + (size_t)bhk * Lk * D, k_i8 + (size_t)bhk * Lk * D,
-                         k_scale + (size_t)bhk * nkb, kb, kb1, Lk, m8, red);
+                         k_scale + (size_t)bhk * nkb, kb, kb1, Lkb, m8, red);
 }
 
 // ------------------------------------------------------------- launcher
@@ -341,7 +349,8 @@ static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* laun
   cfg.numAttrs = 1;
   cudaError_t e = cudaLaunchKernelEx(&cfg, kern, a.q, a.k, a.q_i8, a.k_i8, a.q_scale, a.k_scale,
                                      a.k_mean, BHkv, a.Lq, a.Lk, nqb, nkb, kb_per_cta,
-                                     (int)n_k_ctas, (int)n_q_blocks, a.c);
+                                     (int)n_k_ctas, (int)n_q_blocks, a.c, a.seqlens_q,
+                                     a.seqlens_k, a.H, a.Hkv);
   *launches += 1;
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

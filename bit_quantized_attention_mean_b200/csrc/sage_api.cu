@@ -127,6 +127,16 @@ sage_status sage_quant_qk_qblock(const void* q, const void* k, int8_t* q_i8, int
                                  float* q_scale, float* k_scale, float* k_mean, int B, int H,
                                  int Hkv, int Lq, int Lk, int d, float sm_scale, int q_block_rows,
                                  void* workspace, size_t workspace_bytes, void* stream) {
+  return sage_quant_qk_varlen(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, nullptr, nullptr, B, H,
+                              Hkv, Lq, Lk, d, sm_scale, q_block_rows, workspace, workspace_bytes,
+                              stream);
+}
+
+sage_status sage_quant_qk_varlen(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8,
+                                 float* q_scale, float* k_scale, float* k_mean,
+                                 const int* seqlens_q, const int* seqlens_k, int B, int H,
+                                 int Hkv, int Lq, int Lk, int d, float sm_scale, int q_block_rows,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
@@ -146,7 +156,7 @@ sage_status sage_quant_qk_qblock(const void* q, const void* k, int8_t* q_i8, int
   if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
   sage::QuantArgs a{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
                     q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale),
-                    q_block_rows};
+                    q_block_rows, seqlens_q, seqlens_k};
   int launches = 0;
   cudaError_t e = sage::launch_quant(a, s, &launches);
   if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
@@ -174,6 +184,16 @@ sage_status sage_attn_fwd_prequant_ex(const int8_t* q_i8, const int8_t* k_i8,
                                       const float* q_scale, const float* k_scale, const void* v,
                                       void* out, int B, int H, int Hkv, int Lq, int Lk, int d,
                                       int causal, int q_block_rows, unsigned flags, void* stream) {
+  return sage_attn_fwd_prequant_varlen(q_i8, k_i8, q_scale, k_scale, v, out, nullptr, nullptr, B,
+                                       H, Hkv, Lq, Lk, d, causal, q_block_rows, flags, stream);
+}
+
+sage_status sage_attn_fwd_prequant_varlen(const int8_t* q_i8, const int8_t* k_i8,
+                                          const float* q_scale, const float* k_scale,
+                                          const void* v, void* out, const int* seqlens_q,
+                                          const int* seqlens_k, int B, int H, int Hkv, int Lq,
+                                          int Lk, int d, int causal, int q_block_rows,
+                                          unsigned flags, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
@@ -188,6 +208,8 @@ sage_status sage_attn_fwd_prequant_ex(const int8_t* q_i8, const int8_t* k_i8,
   sage::AttnArgs a{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                    static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1, q_block_rows,
                    (flags & SAGE_PV_ACCUM_F16) != 0u};
+  a.seqlens_q = seqlens_q;
+  a.seqlens_k = seqlens_k;
   int launches = 0;
   cudaError_t e = sage::launch_attn(a, static_cast<cudaStream_t>(stream), &launches);
   g_last_launches = launches;
@@ -211,11 +233,21 @@ sage_status sage_attn_fwd_qblock(const void* q, const void* k, const void* v, vo
 sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* out, int B, int H,
                              int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
                              int q_block_rows, unsigned flags, void* stream) {
+  return sage_attn_fwd_varlen(q, k, v, out, nullptr, nullptr, B, H, Hkv, Lq, Lk, d, causal,
+                              sm_scale, q_block_rows, flags, stream);
+}
+
+sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, void* out,
+                                 const int* seqlens_q, const int* seqlens_k, int B, int H,
+                                 int Hkv, int Lq, int Lk, int d, int causal, float sm_scale,
+                                 int q_block_rows, unsigned flags, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!valid_flags(flags)) return SAGE_ERR_INVALID_ARG;
+  // the V channel maxima of the FP8 path span all Lk positions, padding included
+  if ((seqlens_q || seqlens_k) && flags == SAGE_PV_FP8) return SAGE_ERR_UNSUPPORTED;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return SAGE_ERR_INVALID_ARG;
@@ -240,7 +272,7 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
   float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
   sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
                      q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
-                     fold_constant(sm_scale), q_block_rows};
+                     fold_constant(sm_scale), q_block_rows, seqlens_q, seqlens_k};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
   uint8_t* v8t = reinterpret_cast<uint8_t*>(ws + v8_off);
@@ -252,6 +284,8 @@ sage_status sage_attn_fwd_ex(const void* q, const void* k, const void* v, void* 
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                       static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,
                       q_block_rows, flags == SAGE_PV_ACCUM_F16};
+    aa.seqlens_q = seqlens_q;
+    aa.seqlens_k = seqlens_k;
     if (fp8) {
       aa.pv_fp8 = true;
       aa.v8t = v8t;

@@ -25,6 +25,9 @@ struct QuantArgs {
   int B, H, Hkv, Lq, Lk, d;
   float c;          // fl32(double(sm_scale) * log2(e)), folded into q_scale
   int q_block_rows; // rows per Q quantization block: 128, 64, 32 or 1
+  // padded batches: rows / keys per batch entry ([B], <= Lq / Lk), or null
+  const int* seqlens_q = nullptr;
+  const int* seqlens_k = nullptr;
 };
 
 struct AttnArgs {
@@ -41,6 +44,9 @@ struct AttnArgs {
   bool pv_fp8 = false;            // P and V in E4M3 (v8t, v_scale below; v unused)
   const uint8_t* v8t = nullptr;   // E4M3 V^T [B, Hkv, d, 64 * ceil(Lk / 64)]
   const float* v_scale = nullptr; // [B, Hkv, d]
+  // padded batches: rows / keys per batch entry ([B], <= Lq / Lk), or null
+  const int* seqlens_q = nullptr;
+  const int* seqlens_k = nullptr;
 };
 
 size_t quant_v_fp8_workspace_bytes(int B, int Hkv, int d);

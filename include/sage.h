@@ -199,6 +199,52 @@ SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t 
                                    int causal, int q_block_rows, unsigned flags, void *stream);
 
 /*
+ * sage_quant_qk_varlen / sage_attn_fwd_prequant_varlen / sage_attn_fwd_varlen
+ * -- the _qblock / _ex calls on a padded batch whose entries hold different
+ * numbers of query rows and keys.  Entry b uses rows [0, seqlens_q[b]) of its
+ * [Lq, d] Q rows and keys [0, seqlens_k[b]) of its [Lk, d] K/V rows
+ * (seqlens_q, seqlens_k: device int32 [B], values clamped to [0, Lq] and
+ * [0, Lk]; either pointer may be NULL, meaning every entry uses all Lq rows or
+ * all Lk keys).  Each entry is then computed exactly as the same call on that
+ * entry alone with Lq = seqlens_q[b], Lk = seqlens_k[b]: K smoothing
+ * (step 1 of the SageAttention article's method) subtracts the mean over the
+ * entry's own keys, the last Q and K blocks of an entry are ragged, causal
+ * masking is bottom-right aligned to (seqlens_q[b], seqlens_k[b]).
+ *
+ * Padding is not read and not written by the quantization (its int8 rows and
+ * scales keep whatever the buffers held).  The attention kernels write zeros
+ * to the output rows past seqlens_q[b] and never give weight to a key past
+ * seqlens_k[b]; V rows in [seqlens_k[b], 64 * ceil(seqlens_k[b] / 64)), the
+ * rest of an entry's last 64-key tile, are multiplied by zero weights and
+ * must therefore hold finite values (zeros, say): an Inf or NaN there turns
+ * the entry's output into NaN.  An entry with no rows or no keys outputs
+ * zeros.
+ *
+ * flags: as sage_attn_fwd_ex / sage_attn_fwd_prequant_ex, except that
+ * SAGE_PV_FP8 returns SAGE_ERR_UNSUPPORTED here when either length array is
+ * given (its per-channel V scales span every position, padding included).
+ * Every other argument, layout, error and scratch rule: as the call named.
+ */
+SAGE_API sage_status sage_quant_qk_varlen(const void *q, const void *k,
+                          int8_t *q_i8, int8_t *k_i8,
+                          float *q_scale, float *k_scale, float *k_mean,
+                          const int *seqlens_q, const int *seqlens_k,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          float sm_scale, int q_block_rows,
+                          void *workspace, size_t workspace_bytes, void *stream);
+SAGE_API sage_status sage_attn_fwd_prequant_varlen(const int8_t *q_i8, const int8_t *k_i8,
+                                   const float *q_scale, const float *k_scale,
+                                   const void *v, void *out,
+                                   const int *seqlens_q, const int *seqlens_k,
+                                   int B, int H, int Hkv, int Lq, int Lk, int d,
+                                   int causal, int q_block_rows, unsigned flags, void *stream);
+SAGE_API sage_status sage_attn_fwd_varlen(const void *q, const void *k, const void *v,
+                          void *out, const int *seqlens_q, const int *seqlens_k,
+                          int B, int H, int Hkv, int Lq, int Lk, int d,
+                          int causal, float sm_scale, int q_block_rows, unsigned flags,
+                          void *stream);
+
+/*
  * sage_quant_v_fp8 -- V to FP8 E4M3 with one scale per channel over all Lk
  * tokens of a (batch, kv head): a = max_t |V[t, c]|, r = fl32(448 / a),
  * code = e4m3(fl32(V * r)) (round to nearest even, saturating at 448),
