@@ -55,8 +55,8 @@ INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "264cb6064cf745b1", "workload": "llm-causal-B1H32L4096d128",
-               "bytes_per_launch": 69615872 + 8452608}
+NCU_TRAFFIC = {"attn_sha": "e6eb78fe668b05d5", "workload": "llm-causal-B1H32L4096d128",
+               "bytes_per_launch": 68433920 + 7781632}
 # Same for the decoding kernel (decode.cu + PTX wrappers) on the --decode shape.
 DECODE_NCU_TRAFFIC = {"sha": "35415021c0bda242", "bytes_per_launch": 805530880 + 3755520}
 
