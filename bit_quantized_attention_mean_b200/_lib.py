@@ -375,8 +375,9 @@ def sage_attn_fwd_varlen(q, k, v, out, seqlens_q, seqlens_k, causal, sm_scale, q
                          pv_accum="f32", stream=None):
     """The whole forward pass on a padded batch: entry b attends with its
     first seqlens_q[b] rows over its first seqlens_k[b] keys, exactly as the
-    same call on that entry alone; padding output rows are zeros and the V
-    padding inside an entry's last 64-key tile must be finite."""
+    same call on that entry alone; padding output rows are zeros and (for
+    pv_accum "f32" / "f16") the V padding inside an entry's last 64-key tile
+    must be finite."""
     import torch
     _check_qbr(q_block_rows)
     flags = _flags(pv_accum)

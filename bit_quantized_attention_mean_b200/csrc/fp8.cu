@@ -14,6 +14,10 @@
 // tokens and merging into the global maxima with an integer atomicMax on the
 // fp16 magnitude bits (exact and order-independent); (2) quantization and
 // transposition of 64 x 64 tiles through shared memory.
+//
+// In a padded batch (per-entry key counts Lkb <= Lk) the maxima span the
+// entry's own tokens only and every code past Lkb is 0, so V's padding is
+// never read.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -28,11 +32,13 @@ constexpr int kAmaxTokens = 256;  // tokens per CTA of the maxima pass
 // Largest |V| per channel, as fp16 magnitude bits, into amax[bh * d + c].
 template <int D>
 __global__ void __launch_bounds__(256)
-v_amax_kernel(const __half* __restrict__ v, unsigned* __restrict__ amax, int Lk, int nchunk) {
+v_amax_kernel(const __half* __restrict__ v, unsigned* __restrict__ amax, int Lk, int nchunk,
+              const int* __restrict__ seqlens_k, int Hkv) {
   constexpr int TPR = D / 8;           // 16-byte vectors per token row
   constexpr int RPP = 256 / TPR;       // token rows per pass
   const int bh = blockIdx.x / nchunk, ch = blockIdx.x - bh * nchunk;
-  const int t0 = ch * kAmaxTokens, t1 = min(Lk, t0 + kAmaxTokens);
+  const int Lkb = seqlens_k ? min(max(__ldg(seqlens_k + bh / Hkv), 0), Lk) : Lk;
+  const int t0 = ch * kAmaxTokens, t1 = min(Lkb, t0 + kAmaxTokens);
   const int cg = threadIdx.x % TPR, rr = threadIdx.x / TPR;
   const uint4* base = reinterpret_cast<const uint4*>(v + (size_t)bh * Lk * D) + cg;
   uint32_t m[4] = {0u, 0u, 0u, 0u};  // two channels per word
@@ -63,12 +69,14 @@ v_amax_kernel(const __half* __restrict__ v, unsigned* __restrict__ amax, int Lk,
 template <int D>
 __global__ void __launch_bounds__(256)
 v_fp8_kernel(const __half* __restrict__ v, const unsigned* __restrict__ amax,
-             uint8_t* __restrict__ v8t, float* __restrict__ v_scale, int Lk, int ntt) {
+             uint8_t* __restrict__ v8t, float* __restrict__ v_scale, int Lk, int ntt,
+             const int* __restrict__ seqlens_k, int Hkv) {
   constexpr int CT = D / 64;  // channel tiles per head
   const int tt = blockIdx.x % ntt, rest = blockIdx.x / ntt;
   const int ct = rest % CT, bh = rest / CT;
   const int t0 = tt * 64, c0 = ct * 64;
-  const int rows = min(64, Lk - t0);
+  const int Lkb = seqlens_k ? min(max(__ldg(seqlens_k + bh / Hkv), 0), Lk) : Lk;
+  const int rows = min(64, Lkb - t0);  // <= 0: a tile of padding, all codes 0
   const size_t Lkp = (size_t)ntt * 64;
   __shared__ __half tile[64][64 + 8];  // [token][channel], padded rows
   __shared__ uint32_t codes[64][17];   // [channel][4-token word], padded rows
@@ -119,7 +127,7 @@ size_t quant_v_fp8_workspace_bytes(int B, int Hkv, int d) {
 template <int D>
 static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8t, float* v_scale,
                                         void* workspace, int B, int Hkv, int Lk,
-                                        cudaStream_t st, int* launches) {
+                                        const int* seqlens_k, cudaStream_t st, int* launches) {
   unsigned* amax = static_cast<unsigned*>(workspace);
   cudaError_t e = cudaMemsetAsync(amax, 0, (size_t)B * Hkv * D * sizeof(unsigned), st);
   if (e != cudaSuccess) return e;
@@ -128,19 +136,22 @@ static cudaError_t launch_quant_v_fp8_d(const __half* v, uint8_t* v8t, float* v_
   const int ntt = (Lk + 63) / 64;
   if (BH * nchunk > 0x7fffffffLL || BH * (D / 64) * ntt > 0x7fffffffLL)
     return cudaErrorInvalidConfiguration;
-  v_amax_kernel<D><<<(unsigned)(BH * nchunk), 256, 0, st>>>(v, amax, Lk, nchunk);
+  v_amax_kernel<D><<<(unsigned)(BH * nchunk), 256, 0, st>>>(v, amax, Lk, nchunk, seqlens_k, Hkv);
   *launches += 1;
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   v_fp8_kernel<D><<<(unsigned)(BH * (D / 64) * ntt), 256, 0, st>>>(v, amax, v8t, v_scale, Lk,
-                                                                    ntt);
+                                                                    ntt, seqlens_k, Hkv);
   *launches += 1;
   return cudaGetLastError();
 }
 
 cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8t, float* v_scale, void* workspace,
-                               int B, int Hkv, int Lk, int d, cudaStream_t st, int* launches) {
-  return d == 128 ? launch_quant_v_fp8_d<128>(v, v8t, v_scale, workspace, B, Hkv, Lk, st, launches)
-                  : launch_quant_v_fp8_d<64>(v, v8t, v_scale, workspace, B, Hkv, Lk, st, launches);
+                               int B, int Hkv, int Lk, int d, cudaStream_t st, int* launches,
+                               const int* seqlens_k) {
+  return d == 128 ? launch_quant_v_fp8_d<128>(v, v8t, v_scale, workspace, B, Hkv, Lk, seqlens_k,
+                                              st, launches)
+                  : launch_quant_v_fp8_d<64>(v, v8t, v_scale, workspace, B, Hkv, Lk, seqlens_k,
+                                             st, launches);
 }
 
 }  // namespace sage

@@ -246,8 +246,6 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
   if (st != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!valid_flags(flags)) return SAGE_ERR_INVALID_ARG;
-  // the V channel maxima of the FP8 path span all Lk positions, padding included
-  if ((seqlens_q || seqlens_k) && flags == SAGE_PV_FP8) return SAGE_ERR_UNSUPPORTED;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
     return SAGE_ERR_INVALID_ARG;
@@ -279,7 +277,7 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
   float* v_scale = reinterpret_cast<float*>(ws + vs_off);
   if (e == cudaSuccess && fp8)
     e = sage::launch_quant_v_fp8(static_cast<const __half*>(v), v8t, v_scale, ws + vm_off, B, Hkv,
-                                 Lk, d, s, &launches);
+                                 Lk, d, s, &launches, seqlens_k);
   if (e == cudaSuccess) {
     sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, static_cast<const __half*>(v),
                       static_cast<__half*>(out), B, H, Hkv, Lq, Lk, d, causal == 1,

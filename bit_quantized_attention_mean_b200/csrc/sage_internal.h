@@ -50,8 +50,11 @@ struct AttnArgs {
 };
 
 size_t quant_v_fp8_workspace_bytes(int B, int Hkv, int d);
+// seqlens_k (device int32 [B], or null): per-entry key counts of a padded
+// batch; maxima over each entry's own keys, codes past its count 0
 cudaError_t launch_quant_v_fp8(const __half* v, uint8_t* v8t, float* v_scale, void* workspace,
-                               int B, int Hkv, int Lk, int d, cudaStream_t st, int* launches);
+                               int B, int Hkv, int Lk, int d, cudaStream_t st, int* launches,
+                               const int* seqlens_k = nullptr);
 
 inline bool valid_q_block_rows(int r) { return r == 128 || r == 64 || r == 32 || r == 1; }
 

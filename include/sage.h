@@ -214,15 +214,16 @@ SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t 
  * Padding is not read and not written by the quantization (its int8 rows and
  * scales keep whatever the buffers held).  The attention kernels write zeros
  * to the output rows past seqlens_q[b] and never give weight to a key past
- * seqlens_k[b]; V rows in [seqlens_k[b], 64 * ceil(seqlens_k[b] / 64)), the
- * rest of an entry's last 64-key tile, are multiplied by zero weights and
- * must therefore hold finite values (zeros, say): an Inf or NaN there turns
- * the entry's output into NaN.  An entry with no rows or no keys outputs
+ * seqlens_k[b].  On the fp16 P V paths, V rows in
+ * [seqlens_k[b], 64 * ceil(seqlens_k[b] / 64)), the rest of an entry's last
+ * 64-key tile, are multiplied by zero weights and must therefore hold finite
+ * values (zeros, say): an Inf or NaN there turns the entry's output into NaN.  An entry with no rows or no keys outputs
  * zeros.
  *
- * flags: as sage_attn_fwd_ex / sage_attn_fwd_prequant_ex, except that
- * SAGE_PV_FP8 returns SAGE_ERR_UNSUPPORTED here when either length array is
- * given (its per-channel V scales span every position, padding included).
+ * flags: as sage_attn_fwd_ex / sage_attn_fwd_prequant_ex.  With SAGE_PV_FP8
+ * (sage_attn_fwd_varlen only) each entry's per-channel V scales span its own
+ * keys and the E4M3 codes past seqlens_k[b] are 0, so on that path V's
+ * padding is never read and need not be finite.
  * Every other argument, layout, error and scratch rule: as the call named.
  */
 SAGE_API sage_status sage_quant_qk_varlen(const void *q, const void *k,

@@ -16,7 +16,7 @@ import oracle
 import bit_quantized_attention_mean_b200 as sage
 from bit_quantized_attention_mean_b200 import inputs
 
-from test_gpu_parity import assert_close, assert_quant_bitexact, to_dev, torch_mod
+from test_gpu_parity import assert_close, assert_quant_bitexact, cos, to_dev, torch_mod
 
 pytestmark = pytest.mark.gpu
 
@@ -159,7 +159,41 @@ def test_prequant_varlen_matches_whole_path():
     assert torch.equal(o1, o2)
 
 
-def test_varlen_fp8_is_unsupported_and_bad_args_rejected():
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("case", CASES)
+def test_fp8_varlen_against_oracle(case, causal):
+    """FP8 P V on a padded batch: each entry's V channel scales span its own
+    keys (the oracle quantizes the entry's slice), the codes past its length
+    are 0, so even NaN padding inside the last key tile is harmless here.
+    Bound and cosine gate as the dense FP8 tests: P is rounded at a
+    different point (running vs exact max), by at most half an E4M3 unit."""
+    B, H, Hkv, Lq, Lk, d, lq, lk = case
+    q, k, v = padded_inputs(B, H, Hkv, Lq, Lk, d, lq, lk, seed=5 * Lk + causal)
+    for b in range(B):
+        v[b, :, lk[b]:] = np.nan
+    sm = float(np.float32(1 / math.sqrt(d)))
+    out = sage.attention_varlen(to_dev(q), to_dev(k), to_dev(v), seqlens(lq), seqlens(lk),
+                                causal, sm, pv_accum="fp8")
+    sage.sage_check_device_status()
+    got = out.cpu().numpy().astype(np.float64)
+    for b in range(B):
+        assert np.all(got[b, :, lq[b]:] == 0), f"padding rows of entry {b}"
+        if lq[b] == 0 or lk[b] == 0:
+            assert np.all(got[b] == 0)
+            continue
+        qb, kb, vb = q[b:b + 1, :, :lq[b]], k[b:b + 1, :, :lk[b]], v[b:b + 1, :, :lk[b]]
+        qk = oracle.quant_qk(qb, kb, sm)
+        v8t, vs = oracle.quant_v_fp8(vb)
+        sim = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, causal)
+        g = got[b:b + 1, :, :lq[b]]
+        assert np.all(np.isfinite(g)), f"entry {b}"
+        bound = 2.0 ** -3 * float(np.abs(vb.astype(np.float64)).max()) + 1e-2
+        assert np.abs(g - sim).max() <= bound, f"{case} entry {b}"
+        if np.abs(sim).max() > 0:
+            assert cos(g, sim) >= 0.999, f"{case} entry {b}"
+
+
+def test_varlen_bad_args_rejected():
     torch = torch_mod()
     lib = sage.load_library()
     P = ctypes.c_void_p
@@ -168,14 +202,17 @@ def test_varlen_fp8_is_unsupported_and_bad_args_rejected():
     out = torch.empty_like(q)
     sl = seqlens([64, 10])
     args = (P(q.data_ptr()), P(q.data_ptr()), P(q.data_ptr()), P(out.data_ptr()))
-    st = lib.sage_attn_fwd_varlen(*args, P(sl.data_ptr()), P(0), 2, 2, 2, 64, 64, 64, 0, 0.125,
-                                  128, sage.SAGE_PV_FP8, s)
-    assert st == 2   # SAGE_ERR_UNSUPPORTED
     st = lib.sage_attn_fwd_varlen(*args, P(0), P(sl.data_ptr()), 2, 2, 2, 64, 64, 64, 0, 0.125,
                                   7, 0, s)
     assert st == 1   # bad q_block_rows
-    # without length arrays FP8 stays available
-    st = lib.sage_attn_fwd_varlen(*args, P(0), P(0), 2, 2, 2, 64, 64, 64, 0, 0.125, 128,
-                                  sage.SAGE_PV_FP8, s)
-    assert st == 0
+    st = lib.sage_attn_fwd_varlen(*args, P(0), P(sl.data_ptr()), 2, 2, 2, 64, 64, 64, 0, 0.125,
+                                  128, 3, s)
+    assert st == 1   # both P V variants at once
+    qi = torch.zeros((2, 2, 64, 64), dtype=torch.int8, device="cuda")
+    sc = torch.zeros(8, dtype=torch.float32, device="cuda")
+    st = lib.sage_attn_fwd_prequant_varlen(P(qi.data_ptr()), P(qi.data_ptr()), P(sc.data_ptr()),
+                                           P(sc.data_ptr()), P(q.data_ptr()), P(out.data_ptr()),
+                                           P(sl.data_ptr()), P(sl.data_ptr()), 2, 2, 2, 64, 64,
+                                           64, 0, 128, sage.SAGE_PV_FP8, s)
+    assert st == 1   # the prequant call takes fp16 V
     sage.sage_check_device_status()
