@@ -52,6 +52,9 @@ METRIC = "quantized attention fwd TOPS at 1 B200 and % of INT8/FP16 tensor roofl
 DEFAULT_WORKLOAD = 2
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
+# B200 datasheet dense peaks (TFLOP/s, per GPU) and the exp2 unit's rate
+DATASHEET_TFLOPS = {"int8": 4500.0, "fp8": 4500.0, "fp16": 2250.0}
+EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per clock per SM (measured 15.9)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
@@ -164,6 +167,27 @@ class ClockSampler:
         reasons = [n for bit, n in self.REASONS.items() if mask & bit and n != "gpu_idle"]
         return {"sm_mhz": statistics.median([s[0] for s in busy]) if busy else None,
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(busy)}
+
+
+def secondary_ceilings(d, pairs, attn_ms, t_roof_ms, fp8, sms, sm_mhz):
+    """The two further bars of the attention kernel: the fraction of the
+    datasheet dense peaks (QK at INT8, P V at FP16 or FP8), and the exp2
+    ceiling -- one ex2 per unmasked pair on the SMs' ex2 units at the SM
+    clock seen during the run -- as its time, the highest fraction of the
+    (measured) combined roofline it leaves reachable, and how close the
+    kernel comes to it."""
+    pv = DATASHEET_TFLOPS["fp8" if fp8 else "fp16"]
+    t_nom_ms = (2.0 * d * pairs / (DATASHEET_TFLOPS["int8"] * 1e12)
+                + 2.0 * d * pairs / (pv * 1e12)) * 1e3
+    t_exp2_ms = pairs / (EX2_PER_CLK_PER_SM * sms * sm_mhz * 1e6) * 1e3
+    return {
+        "datasheet": {"frac": t_nom_ms / attn_ms, "t_roof_ms": t_nom_ms,
+                      "peaks_tflops": {"qk_int8": DATASHEET_TFLOPS["int8"],
+                                       "pv": pv}},
+        "exp2": {"t_ms": t_exp2_ms, "max_roofline_frac": min(1.0, t_roof_ms / t_exp2_ms),
+                 "frac_of_ceiling": t_exp2_ms / attn_ms, "sms": sms, "sm_mhz": sm_mhz,
+                 "ex2_per_clk_per_sm": EX2_PER_CLK_PER_SM},
+    }
 
 
 # ---------------------------------------------------------- distributed
@@ -396,6 +420,7 @@ def run_ours(args, w):
 
     result = None
     if rank == 0:
+        clk = clocks.summary()
         ops = 4.0 * d * w.pairs()
         ms_per_step = total_ms / n
         value = weak_scaling_value(ops, world, ms_per_step)
@@ -430,12 +455,16 @@ def run_ours(args, w):
                                        f"TFLOP/s ({peaks.get('source')} bf16 burst), P_int8 = "
                                        f"{INT8_OVER_FP16} x P_fp16 (nominal ratio)")},
             "kernel_ms": {"attention": attn_avg_ms, "quant": quant_avg_ms},
+            "ceilings": secondary_ceilings(
+                d, w.pairs(), attn_avg_ms, t_roof_ms, fp8,
+                torch.cuda.get_device_properties(dev).multi_processor_count,
+                clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0),
             "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
             "e2e": {"value": weak_scaling_value(ops, world, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": int(qn.nbytes + kn.nbytes + vn.nbytes),
                     "d2h_bytes_per_step": int(qn.nbytes)},
             "gpu_launches": n_launches,
-            "clocks": clocks.summary(),
+            "clocks": clk,
         }
     if world > 1:
         torch.distributed.barrier()

@@ -78,3 +78,23 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["unit"] == "TOPS" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_secondary_ceilings_arithmetic():
+    """Closed forms: the LLM workload's 268,451,840 causal pairs at d = 128."""
+    import bench
+    pairs = 32 * 4096 * 4097 // 2
+    c = bench.secondary_ceilings(128, pairs, attn_ms=0.1, t_roof_ms=0.05, fp8=False,
+                                 sms=148, sm_mhz=1965.0)
+    t_nom = (256 * pairs / 4.5e15 + 256 * pairs / 2.25e15) * 1e3
+    assert c["datasheet"]["t_roof_ms"] == pytest.approx(t_nom)
+    assert c["datasheet"]["frac"] == pytest.approx(t_nom / 0.1)
+    t_exp2 = pairs / (16 * 148 * 1965e6) * 1e3          # ~0.0577 ms
+    assert c["exp2"]["t_ms"] == pytest.approx(t_exp2)
+    assert c["exp2"]["max_roofline_frac"] == pytest.approx(0.05 / t_exp2)
+    assert c["exp2"]["frac_of_ceiling"] == pytest.approx(t_exp2 / 0.1)
+    # FP8 P V is charged at the 8-bit datasheet rate; a roofline longer than
+    # the exp2 time leaves the full fraction reachable
+    c8 = bench.secondary_ceilings(128, pairs, 0.1, 1.0, True, 148, 1965.0)
+    assert c8["datasheet"]["t_roof_ms"] == pytest.approx(512 * pairs / 4.5e15 * 1e3)
+    assert c8["exp2"]["max_roofline_frac"] == 1.0
