@@ -13,6 +13,7 @@ Exported names mirror the C ABI:
     sage_attn_decode, sage_attn_decode_prequant, sage_attn_decode_workspace_size,
     sage_quant_v_fp8, sage_quant_v_fp8_workspace_size, sage_attn_fwd_prequant_fp8pv,
     sage_quant_qk_varlen, sage_attn_fwd_prequant_varlen, sage_attn_fwd_varlen,
+    sage_quant_k,
     sage_quant_workspace_size, sage_attn_workspace_size,
     sage_check_device_status, sage_status_string, sage_last_launch_count
 plus conveniences that allocate outputs: ``quant_qk``, ``attention``,
@@ -62,4 +63,5 @@ from ._lib import (  # noqa: F401
     sage_attn_fwd_prequant_varlen,
     sage_attn_fwd_varlen,
     attention_varlen,
+    sage_quant_k,
 )

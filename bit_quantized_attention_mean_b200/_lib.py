@@ -44,6 +44,7 @@ SYMBOLS = (
     "sage_quant_qk_varlen",
     "sage_attn_fwd_prequant_varlen",
     "sage_attn_fwd_varlen",
+    "sage_quant_k",
 )
 
 Q_BLOCK_ROWS = (128, 64, 32, 1)  # accepted Q quantization block heights
@@ -136,6 +137,8 @@ def load_library():
         lib.sage_attn_fwd_prequant_varlen.restype = I
         lib.sage_attn_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P]
         lib.sage_attn_fwd_varlen.restype = I
+        lib.sage_quant_k.argtypes = [P, P, P, P, I, I, I, I, P, Z, P]
+        lib.sage_quant_k.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
         _lib = lib
@@ -389,6 +392,18 @@ def sage_attn_fwd_varlen(q, k, v, out, seqlens_q, seqlens_k, causal, sm_scale, q
         _seqlens(seqlens_q, "seqlens_q", B), _seqlens(seqlens_k, "seqlens_k", B),
         B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows), flags,
         _stream(stream)), "sage_attn_fwd_varlen")
+
+
+def sage_quant_k(k, k_i8, k_scale, k_mean, workspace=None, stream=None):
+    """Smooth K and quantize it in 64-row blocks (the K half of
+    sage_quant_qk) into the given output tensors."""
+    import torch
+    B, Hkv, Lk, d = k.shape
+    _check(load_library().sage_quant_k(
+        _dev(k, torch.float16, "k"), _dev(k_i8, torch.int8, "k_i8", k.shape),
+        _dev(k_scale, torch.float32, "k_scale", (B, Hkv, -(-Lk // 64))),
+        _dev(k_mean, torch.float32, "k_mean", (B, Hkv, d)), B, Hkv, Lk, d,
+        *_workspace(workspace), _stream(stream)), "sage_quant_k")
 
 
 def sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:

@@ -331,7 +331,7 @@ static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* laun
   if ((long long)kb_per_cta * SAGE_K_BLOCK_ROWS / (kQuantThreads / (D / 8)) > 8192)
     return cudaErrorInvalidValue;
   const long long n_k_ctas = (long long)BHkv * cl;
-  const long long n_q_blocks = (long long)BH * nqb;
+  const long long n_q_blocks = a.skip_q ? 0 : (long long)BH * nqb;
   const long long n_q_ctas = (n_q_blocks + cl - 1) / cl * cl;
   if (n_k_ctas + n_q_ctas > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
 

@@ -296,6 +296,32 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
 
+sage_status sage_quant_k(const void* k, int8_t* k_i8, float* k_scale, float* k_mean, int B,
+                         int Hkv, int Lk, int d, void* workspace, size_t workspace_bytes,
+                         void* stream) {
+  g_last_launches = 0;
+  sage_status st = check_shape(B, Hkv, Hkv, 1, Lk, d);
+  if (st != SAGE_OK) return st;
+  if (!k || !k_i8 || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(k_i8) || !aligned16(k_scale) || !aligned16(k_mean))
+    return SAGE_ERR_INVALID_ARG;
+  const size_t need = sage::quant_workspace_bytes(B, Hkv, Lk, d);
+  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* ws = workspace;
+  const bool own = !ws && need > 0;
+  if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
+  sage::QuantArgs a{nullptr, static_cast<const __half*>(k), nullptr, k_i8, nullptr, k_scale,
+                    k_mean, ws, B, Hkv, Hkv, 1, Lk, d, 1.f, SAGE_Q_BLOCK};
+  a.skip_q = true;
+  int launches = 0;
+  cudaError_t e = sage::launch_quant(a, s, &launches);
+  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
+  g_last_launches = launches;
+  return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
+}
+
 size_t sage_attn_decode_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
   if (check_shape(B, H, Hkv, Lq, Lk, d) != SAGE_OK || (long long)(H / Hkv) * Lq > 128) return 0;
   const sage::DecodePlan p = sage::decode_plan(B, H, Hkv, Lq, Lk, d);

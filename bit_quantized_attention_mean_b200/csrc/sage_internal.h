@@ -28,6 +28,8 @@ struct QuantArgs {
   // padded batches: rows / keys per batch entry ([B], <= Lq / Lk), or null
   const int* seqlens_q = nullptr;
   const int* seqlens_k = nullptr;
+  // K only (smoothing + K blocks); the Q arguments are not used
+  bool skip_q = false;
 };
 
 struct AttnArgs {

@@ -117,6 +117,24 @@ SAGE_API sage_status sage_quant_qk_qblock(const void *q, const void *k,
                           float sm_scale, int q_block_rows,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/*
+ * sage_quant_k -- steps 1-2 alone: K smoothing (mean over each (batch, kv
+ * head)'s Lk tokens, the SageAttention article's "对 K 进行平滑处理", method
+ * section) and INT8 quantization of the smoothed K in 64-row blocks, with
+ * the same codes, scales and mean as sage_quant_qk produces for K (one
+ * launch of K clusters only).  For a K that is quantized once and attended
+ * many times, e.g. a key cache for the decoding calls.
+ *   k        fp16 [B, Hkv, Lk, d]          (in)
+ *   k_i8     int8 [B, Hkv, Lk, d]          (out)
+ *   k_scale  fp32 [B, Hkv, ceil(Lk/64)]    (out)
+ *   k_mean   fp32 [B, Hkv, d]              (out)
+ *   workspace, workspace_bytes: as sage_quant_qk (sage_quant_workspace_size).
+ * Errors: as sage_quant_qk.
+ */
+SAGE_API sage_status sage_quant_k(const void *k, int8_t *k_i8, float *k_scale, float *k_mean,
+                          int B, int Hkv, int Lk, int d,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
 /* Bytes of scratch sage_quant_qk needs (currently 0). */
 SAGE_API size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d);
 
