@@ -58,10 +58,10 @@ EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per clock per SM (measured 15.9)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "e6eb78fe668b05d5", "workload": "llm-causal-B1H32L4096d128",
+NCU_TRAFFIC = {"attn_sha": "0426d895995a5473", "workload": "llm-causal-B1H32L4096d128",
                "bytes_per_launch": 68433920 + 7781632}
 # Same for the decoding kernel (decode.cu + PTX wrappers) on the --decode shape.
-DECODE_NCU_TRAFFIC = {"sha": "35415021c0bda242", "bytes_per_launch": 805530880 + 3755520}
+DECODE_NCU_TRAFFIC = {"sha": "6a43014109bd395c", "bytes_per_launch": 805530880 + 3755520}
 
 
 def load_peaks():
@@ -74,26 +74,35 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
+def _code_only(text: bytes) -> bytes:
+    """C/C++ source without its comments and blank lines, so that a comment
+    edit does not invalidate counters taken on unchanged code."""
+    import re
+    t = re.sub(rb"/\*.*?\*/", b"", text, flags=re.S)
+    t = re.sub(rb"//[^\n]*", b"", t)
+    return b"\n".join(ln.rstrip() for ln in t.split(b"\n") if ln.strip())
+
+
 def decode_source_hash():
-    """Hash of the decoding kernel's source and of the PTX wrappers."""
+    """Hash of the decoding kernel's code and of the PTX wrappers."""
     csrc = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc")
     h = hashlib.sha256()
     for name in ("decode.cu", "sm100_ptx.cuh"):
         with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+            h.update(_code_only(f.read()))
     return h.hexdigest()[:16]
 
 
 def attn_source_hash():
     """Hash of the attention kernel's device code (attn.cu up to its host
-    section) and of the PTX wrappers it is built from."""
+    section) and of the PTX wrappers it is built from, comments excluded."""
     csrc = os.path.join(ROOT, "bit_quantized_attention_mean_b200", "csrc")
     with open(os.path.join(csrc, "attn.cu"), "rb") as f:
         text = f.read()
     marker = b"// ------------------------------------------------------------------- host"
-    h = hashlib.sha256(text.split(marker)[0])
+    h = hashlib.sha256(_code_only(text.split(marker)[0]))
     with open(os.path.join(csrc, "sm100_ptx.cuh"), "rb") as f:
-        h.update(f.read())
+        h.update(_code_only(f.read()))
     return h.hexdigest()[:16]
 
 

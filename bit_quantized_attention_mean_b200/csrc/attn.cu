@@ -1,10 +1,11 @@
 // attn.cu -- fused 8-bit attention forward for sm_100a (B200).
 //
-// Follows the SageAttention article, method section: S = Q_i8 K_i8^T with an
-// INT32 accumulator ("对 Q, K 进行分块 INT8 量化"), dequantized by
-// q_scale * k_scale, softmax over FlashAttention-style tiles, and O = P V with
-// P and V in FP16 ("对 P, V 采用 FP16 ...").  sm_scale * log2(e) is already in
-// q_scale, so the softmax runs in base 2 (exp2).
+// Follows the SageAttention article (method section: the per-block INT8
+// quantization step and the FP16 P V step): S = Q_i8 K_i8^T with an INT32
+// accumulator, dequantized by q_scale * k_scale, softmax over
+// FlashAttention-style tiles, and O = P V with P and V in FP16.
+// sm_scale * log2(e) is already in q_scale, so the softmax runs in base 2
+// (exp2).
 //
 // One CTA owns one 128-row Q tile (the Q quantization block) and walks the
 // 64-row K/V tiles (the K quantization block) of its (batch, kv head):
@@ -28,8 +29,8 @@
 // MMAs.  tcgen05 operations from one thread execute in issue order, which is
 // what makes reusing a score buffer for S_{j+2} after P_j V_j safe.
 //
-// F16ACC selects the accumulator the article names for P V ("对 P, V 采用
-// FP16 数据类型的矩阵乘法累加器"): the P V products accumulate in fp16 (one value
+// F16ACC selects the accumulator the article names for P V (an fp16
+// accumulator, method section, FP16 P V step): the P V products accumulate in fp16 (one value
 // per tensor-memory column, in its low half), and the running max is exact
 // (O rescaled whenever it grows) so that P <= 1 keeps the sums in fp16 range.
 // The default accumulates in fp32.

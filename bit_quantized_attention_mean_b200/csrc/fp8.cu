@@ -1,6 +1,6 @@
 // fp8.cu -- V to FP8 (E4M3) with one scale per channel, for the P V product
-// with P and V in FP8 that the SageAttention2 description on the
-// SageAttention pages names ("将 P, V 量化至 FP8").
+// with P and V in FP8 that the SageAttention2 description (the INT4 search
+// results page, SageAttention2 entry) proposes.
 //
 // Per (batch, kv head) and channel c over all Lk tokens: a = max_t |V[t, c]|,
 // r = fl32(448 / a), code = e4m3(fl32(V * r)) rounded to nearest even and

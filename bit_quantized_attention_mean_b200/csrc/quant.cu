@@ -1,6 +1,6 @@
 // quant.cu -- K smoothing and per-block INT8 quantization of Q and K for
-// sm_100a (SageAttention article, method section: "对 K 进行平滑处理" and
-// "对 Q, K 进行分块 INT8 量化").
+// sm_100a (SageAttention article, method section: the K smoothing step and
+// the per-block INT8 quantization step).
 //
 // One launch, HBM-bound.  The grid is made of thread-block clusters of
 // kCluster CTAs (16 when there are few kv heads, so the K work still spreads

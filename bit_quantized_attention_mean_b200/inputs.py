@@ -4,8 +4,8 @@ This module only draws random numbers and casts them to fp16; it holds none of
 the attention or quantization arithmetic.  Both the CUDA path and the CPU
 oracle are fed from here, so that they see byte-identical inputs.
 
-The SageAttention article (section "对 K 进行平滑处理", channel-wise outliers in
-K for image/video models) motivates the per-channel K offsets below; the five
+The SageAttention article (method section, K smoothing step: channel-wise
+outliers in K for image/video models) motivates the per-channel K offsets below; the five
 shapes stand in for the text (LLM, GQA, long-context) and video-diffusion
 workloads the articles talk about.  No public dataset is used.
 

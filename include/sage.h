@@ -119,7 +119,7 @@ SAGE_API sage_status sage_quant_qk_qblock(const void *q, const void *k,
 
 /*
  * sage_quant_k -- steps 1-2 alone: K smoothing (mean over each (batch, kv
- * head)'s Lk tokens, the SageAttention article's "对 K 进行平滑处理", method
+ * head)'s Lk tokens, the SageAttention article's K smoothing step, method
  * section) and INT8 quantization of the smoothed K in 64-row blocks, with
  * the same codes, scales and mean as sage_quant_qk produces for K (one
  * launch of K clusters only).  For a K that is quantized once and attended
@@ -192,16 +192,16 @@ SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const vo
 /*
  * sage_attn_fwd_ex / sage_attn_fwd_prequant_ex -- the _qblock entry points
  * with a flags word.  SAGE_PV_ACCUM_F16 selects the P V accumulator the
- * SageAttention article states ("对 P, V 采用 FP16 数据类型的矩阵乘法累加器",
- * method section): P and V stay fp16 and their products are summed in fp16
+ * SageAttention article states (an fp16 accumulator, method section, FP16
+ * P V step): P and V stay fp16 and their products are summed in fp16
  * (the tensor core's F16 D format) instead of fp32.  With it the running
  * row max is kept exact (O is rescaled whenever it grows), so P <= 1 and, as
  * the article argues, the sums stay within the fp16 range; the result is
  * less accurate than the fp32 default (the error grows with Lk) and no
  * faster on this GPU.  SAGE_PV_FP8 (sage_attn_fwd_ex only) quantizes V to
  * E4M3 per channel (sage_quant_v_fp8) and P to E4M3 and runs P V on the FP8
- * tensor-core path with fp32 sums, as the SageAttention2 description on the
- * same pages states ("将 P, V 量化至 FP8").  flags = 0 is identical to the
+ * tensor-core path with fp32 sums, as the SageAttention2 description (INT4
+ * search results page, SageAttention2 entry) proposes.  flags = 0 is identical to the
  * _qblock calls.  Any other value, both bits together, or SAGE_PV_FP8 given
  * to sage_attn_fwd_prequant_ex (which takes fp16 V; use
  * sage_attn_fwd_prequant_fp8pv) returns SAGE_ERR_INVALID_ARG.

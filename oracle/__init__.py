@@ -7,15 +7,16 @@ only compiles it (gcc, OpenMP, no fast-math, no FMA contraction) and marshals
 numpy arrays through ctypes.
 
 Functions and the passages they follow (SageAttention article, method section):
-  k_mean          K smoothing, "对 K 进行平滑处理"
-  quant_qk        per-block INT8 quantization of Q and smoothed K,
-                  "对 Q, K 进行分块 INT8 量化"
+  k_mean          the K smoothing step
+  quant_qk        the per-block INT8 quantization step, for Q and the
+                  smoothed K
   attn_quant_sim  INT32-accumulated QK^T, dequantization, softmax with P kept
-                  in FP16, "对 P, V 采用 FP16 ..."
-  attn_fp64       plain softmax(QK^T * sm_scale) V in fp64 (the accuracy
-                  baseline the article compares against, "全精度 Attention")
-  e4m3_encode /   the FP8 (E4M3) format of the SageAttention2 description
-  e4m3_decode     ("将 P, V 量化至 FP8"), round to nearest even, saturating
+                  in FP16 (the FP16 P V step)
+  attn_fp64       plain softmax(QK^T * sm_scale) V in fp64 (the full-precision
+                  attention the article measures its accuracy against)
+  e4m3_encode /   the FP8 (E4M3) format for P and V that the SageAttention2
+  e4m3_decode     description (INT4 search results page, SageAttention2 entry)
+                  proposes, round to nearest even, saturating
   quant_v_fp8     V to E4M3 with one scale per channel, stored channel-major
   attn_fp8pv_sim  the forward pass with P and V in E4M3 for the P V product
 """

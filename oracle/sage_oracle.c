@@ -7,11 +7,11 @@
  * share no code, headers, tables or constants.
  *
  * It follows the SageAttention article ("又快又准，即插即用！清华8比特量化
- * Attention"), method section:
- *   - "对 K 进行平滑处理": K <- K - mean(K), which leaves softmax(QK^T) unchanged;
- *   - "对 Q, K 进行分块 INT8 量化": INT8 quantization of Q and K per
- *     FlashAttention-sized block, INT8 matmul with an INT32 accumulator;
- *   - "对 P, V 采用 FP16 数据类型的矩阵乘法累加器": P and V kept in FP16.
+ * Attention"), method section, whose three steps are:
+ *   - K smoothing: K <- K - mean(K), which leaves softmax(QK^T) unchanged;
+ *   - per-block INT8 quantization of Q and K at FlashAttention block size,
+ *     with an INT8 matmul accumulating in INT32;
+ *   - P and V kept in FP16 for the P V product.
  *
  * Readings where the article is silent (each is a plain choice, listed with
  * its reason in the design notes of the repository):
