@@ -138,7 +138,7 @@ class ClockSampler:
             except Exception:
                 self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
-        except Exception as e:  # pragma: no cover - depends on the box
+        except Exception as e:  # pragma: no cover - depends on the machine
             self._nvml = None
             self.error = str(e)
 

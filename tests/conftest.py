@@ -10,7 +10,7 @@ if ROOT not in sys.path:
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
-    config.addinivalue_line("markers", "slow: full-size workload parity (GPU box only)")
+    config.addinivalue_line("markers", "slow: full-size workload parity (needs a B200)")
 
 
 @pytest.fixture(scope="session")
