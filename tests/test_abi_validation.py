@@ -1,0 +1,95 @@
+"""CPU checks of the C ABI's argument validation: every call below carries
+one invalid argument that the library rejects before it touches the device
+(shape, block height, flags, causal flag, sm_scale, null or misaligned
+pointer), so the stated status comes back without a GPU and the dummy
+pointers are never dereferenced."""
+import ctypes
+import math
+
+import pytest
+
+import bit_quantized_attention_mean_b200 as sage
+
+P = ctypes.c_void_p
+A = P(1 << 20)          # a 16-byte aligned dummy address (never dereferenced)
+M = P((1 << 20) + 4)    # misaligned
+N = P(0)                # null
+S = P(0)                # default stream
+OK_, INVALID, UNSUPPORTED = 0, 1, 2
+
+
+def quant_k(k=A, ki=A, ks=A, km=A, B=1, Hkv=2, Lk=128, d=64):
+    return sage.load_library().sage_quant_k(k, ki, ks, km, B, Hkv, Lk, d, N, 0, S)
+
+
+def quant_qk_varlen(q=A, qs=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, sm=0.125, qbr=128):
+    return sage.load_library().sage_quant_qk_varlen(q, A, A, A, qs, A, A, A, A, B, H, Hkv, Lq,
+                                                    Lk, d, sm, qbr, N, 0, S)
+
+
+def fwd_varlen(out=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, causal=0, sm=0.125, qbr=128,
+               flags=0):
+    return sage.load_library().sage_attn_fwd_varlen(A, A, A, out, A, A, B, H, Hkv, Lq, Lk, d,
+                                                    causal, sm, qbr, flags, S)
+
+
+def prequant_varlen(qbr=128, flags=0, causal=0):
+    return sage.load_library().sage_attn_fwd_prequant_varlen(A, A, A, A, A, A, A, A, 1, 2, 2,
+                                                             128, 128, 64, causal, qbr, flags, S)
+
+
+def quant_v_fp8(v8t=A, vs=A, d=64, Lk=128):
+    return sage.load_library().sage_quant_v_fp8(A, v8t, vs, 1, 2, Lk, d, N, 0, S)
+
+
+def decode_varlen(H=8, Hkv=2, Lq=1, causal=0, qbr=1):
+    return sage.load_library().sage_attn_decode_prequant_varlen(A, A, A, A, A, A, A, 1, H, Hkv,
+                                                                Lq, 1024, 128, causal, qbr, N, 0,
+                                                                S)
+
+
+CASES = [
+    ("quant_k: no keys", lambda: quant_k(Lk=0), INVALID),
+    ("quant_k: d = 96", lambda: quant_k(d=96), UNSUPPORTED),
+    ("quant_k: null K", lambda: quant_k(k=N), INVALID),
+    ("quant_k: misaligned k_i8", lambda: quant_k(ki=M), INVALID),
+    ("quant_qk_varlen: sm_scale 0", lambda: quant_qk_varlen(sm=0.0), INVALID),
+    ("quant_qk_varlen: block height 48", lambda: quant_qk_varlen(qbr=48), INVALID),
+    ("quant_qk_varlen: null q_scale", lambda: quant_qk_varlen(qs=N), INVALID),
+    ("quant_qk_varlen: H % Hkv != 0", lambda: quant_qk_varlen(H=3), INVALID),
+    ("fwd_varlen: both P V variants", lambda: fwd_varlen(flags=3), INVALID),
+    ("fwd_varlen: unknown flag", lambda: fwd_varlen(flags=8), INVALID),
+    ("fwd_varlen: causal 2", lambda: fwd_varlen(causal=2), INVALID),
+    ("fwd_varlen: sm_scale inf", lambda: fwd_varlen(sm=math.inf), INVALID),
+    ("fwd_varlen: sm_scale nan", lambda: fwd_varlen(sm=math.nan), INVALID),
+    ("fwd_varlen: d = 80", lambda: fwd_varlen(d=80), UNSUPPORTED),
+    ("fwd_varlen: misaligned out", lambda: fwd_varlen(out=M), INVALID),
+    ("fwd_varlen: no batch", lambda: fwd_varlen(B=0), INVALID),
+    ("prequant_varlen: FP8 takes E4M3 V", lambda: prequant_varlen(flags=sage.SAGE_PV_FP8),
+     INVALID),
+    ("prequant_varlen: block height 0", lambda: prequant_varlen(qbr=0), INVALID),
+    ("prequant_varlen: causal -1", lambda: prequant_varlen(causal=-1), INVALID),
+    ("quant_v_fp8: d = 96", lambda: quant_v_fp8(d=96), UNSUPPORTED),
+    ("quant_v_fp8: null v8t", lambda: quant_v_fp8(v8t=N), INVALID),
+    ("quant_v_fp8: misaligned v_scale", lambda: quant_v_fp8(vs=M), INVALID),
+    ("decode: 16 heads x 9 queries > one tile", lambda: decode_varlen(H=16, Hkv=1, Lq=9),
+     UNSUPPORTED),
+    ("decode: causal 3", lambda: decode_varlen(causal=3), INVALID),
+    ("decode: block height 2", lambda: decode_varlen(qbr=2), INVALID),
+]
+
+
+@pytest.mark.parametrize("what,call,want", CASES, ids=[c[0] for c in CASES])
+def test_rejected_before_the_device(what, call, want):
+    got = call()
+    assert got == want, f"{what}: {sage.sage_status_string(got)}"
+    assert sage.sage_last_launch_count() == 0
+
+
+def test_workspace_sizes_of_the_newer_calls():
+    # FP8 V maxima: one uint32 per (batch, kv head, channel), 256-byte rounded
+    assert sage.sage_quant_v_fp8_workspace_size(2, 4, 128) == 4096
+    assert sage.sage_quant_v_fp8_workspace_size(1, 1, 64) == 256
+    # decoding layout: unsupported shapes report 0
+    assert sage.sage_attn_decode_workspace_size(1, 16, 1, 9, 256, 64) == 0
+    assert sage.sage_attn_decode_workspace_size(1, 8, 8, 1, 256, 96) == 0
