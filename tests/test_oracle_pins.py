@@ -417,6 +417,30 @@ def test_sim_closed_forms(causal):
     np.testing.assert_array_equal(out, ref)
 
 
+@pytest.mark.parametrize("Lq,Lk", [(40, 100), (100, 40), (64, 64), (1, 70)])
+def test_sim_bottom_right_alignment_closed_form(Lq, Lk):
+    """All K rows equal: smoothed K is 0, every visible key gets the same
+    weight, so causal row i is the mean of the first
+    n_i = clamp(i + Lk - Lq + 1, 0, Lk) value rows (0 when n_i = 0), and a
+    non-causal row is the mean of all Lk.  An off-by-one in the mask's
+    alignment, or aligning at the top-left, changes n_i."""
+    B, H, d = 1, 2, 32
+    q, k, v = inputs.make_custom(B, H, H, Lq, Lk, d, seed=Lq * 7 + Lk)
+    ke = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    vv = v.astype(np.float64)
+    csum = np.concatenate([np.zeros((B, H, 1, d)), np.cumsum(vv, axis=2)], axis=2)
+    out, _ = _sim(q, ke, v, True, 0.125)
+    n = np.clip(np.arange(Lq) + Lk - Lq + 1, 0, Lk)
+    ref = np.zeros((B, H, Lq, d))
+    for i in range(Lq):
+        if n[i] > 0:
+            ref[:, :, i] = csum[:, :, n[i]] / n[i]
+    np.testing.assert_allclose(out, ref, rtol=0, atol=1e-12)
+    out, _ = _sim(q, ke, v, False, 0.125)
+    np.testing.assert_allclose(out, np.broadcast_to(csum[:, :, Lk:] / Lk, out.shape),
+                               rtol=0, atol=1e-12)
+
+
 def test_sim_kv_block_permutation_invariance():
     q, k, v = inputs.make_custom(1, 1, 1, 64, 256, 64, seed=51)
     perm = np.array([2, 0, 3, 1])
@@ -553,6 +577,27 @@ def test_fp8pv_sim_closed_forms():
     out_nc = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, False)
     assert np.allclose(out_nc, np.broadcast_to(deq.mean(axis=2, keepdims=True), out_nc.shape),
                        rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("Lq,Lk", [(40, 100), (100, 40)])
+def test_fp8pv_sim_bottom_right_alignment_closed_form(Lq, Lk):
+    """The FP8 simulation's own causal mask, for Lq != Lk: with equal
+    scores (P = 1 exactly in E4M3), row i is the mean of the first
+    clamp(i + Lk - Lq + 1, 0, Lk) dequantized V rows, 0 when there are none."""
+    B, H, d = 1, 2, 64
+    q, k, v = inputs.make_custom(B, H, H, Lq, Lk, d, seed=Lq + 3 * Lk)
+    ke = np.broadcast_to(k[:, :, :1], k.shape).copy()
+    qk = oracle.quant_qk(q, ke, 0.125)
+    v8t, vs = oracle.quant_v_fp8(v)
+    deq = np.swapaxes(np.vectorize(oracle.e4m3_decode)(v8t), 2, 3)[:, :, :Lk] * vs[:, :, None, :]
+    csum = np.concatenate([np.zeros((B, H, 1, d)), np.cumsum(deq, axis=2)], axis=2)
+    out = oracle.attn_fp8pv_sim(*qk[:4], v8t, vs, True)
+    n = np.clip(np.arange(Lq) + Lk - Lq + 1, 0, Lk)
+    ref = np.zeros((B, H, Lq, d))
+    for i in range(Lq):
+        if n[i] > 0:
+            ref[:, :, i] = csum[:, :, n[i]] / n[i]
+    assert np.allclose(out, ref, rtol=1e-12, atol=1e-12)
 
 
 def test_fp8pv_sim_tracks_the_fp16_path_and_gqa():
