@@ -201,8 +201,9 @@ SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const vo
  * faster on this GPU.  SAGE_PV_FP8 (sage_attn_fwd_ex only) quantizes V to
  * E4M3 per channel (sage_quant_v_fp8) and P to E4M3 and runs P V on the FP8
  * tensor-core path with fp32 sums, as the SageAttention2 description (INT4
- * search results page, SageAttention2 entry) proposes.  flags = 0 is identical to the
- * _qblock calls.  Any other value, both bits together, or SAGE_PV_FP8 given
+ * search results page, SageAttention2 entry) proposes.  flags = 0 is
+ * identical to the _qblock calls.  Any other value, both bits together, or
+ * SAGE_PV_FP8 given
  * to sage_attn_fwd_prequant_ex (which takes fp16 V; use
  * sage_attn_fwd_prequant_fp8pv) returns SAGE_ERR_INVALID_ARG.
  */
@@ -235,8 +236,8 @@ SAGE_API sage_status sage_attn_fwd_prequant_ex(const int8_t *q_i8, const int8_t 
  * seqlens_k[b].  On the fp16 P V paths, V rows in
  * [seqlens_k[b], 64 * ceil(seqlens_k[b] / 64)), the rest of an entry's last
  * 64-key tile, are multiplied by zero weights and must therefore hold finite
- * values (zeros, say): an Inf or NaN there turns the entry's output into NaN.  An entry with no rows or no keys outputs
- * zeros.
+ * values (zeros, say): an Inf or NaN there turns the entry's output into
+ * NaN.  An entry with no rows or no keys outputs zeros.
  *
  * flags: as sage_attn_fwd_ex / sage_attn_fwd_prequant_ex.  With SAGE_PV_FP8
  * (sage_attn_fwd_varlen only) each entry's per-channel V scales span its own
