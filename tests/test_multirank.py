@@ -78,6 +78,21 @@ def test_reference_arm_runs_on_rank_zero_only():
     assert line["unit"] == "TOPS" and line["value"] > 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+    for key in ("metric", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+                "vs_baseline", "dtype", "data", "config"):
+        assert key in line, key
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["higher_is_better"] is True
+    assert line["config"]["workload"] == "tiny-noncausal-B1H2L256d64"
+
+
+def test_source_hash_ignores_comments_only():
+    """The key of the recorded ncu traffic: comments and blank lines do not
+    change it, code does."""
+    import bench
+    code = b"int f(int x) {\n  return x + 1;  // one more\n}\n"
+    assert bench._code_only(code) == bench._code_only(
+        b"/* header\n   block */\nint f(int x) {\n\n  return x + 1;\n}\n// end\n")
+    assert bench._code_only(code) != bench._code_only(code.replace(b"x + 1", b"x + 2"))
 
 
 def test_secondary_ceilings_arithmetic():
