@@ -232,6 +232,20 @@ def weak_scaling_value(ops_per_rank, world, ms_per_step):
 
 # ------------------------------------------------------------ CPU oracle
 
+# The one-off CPU baseline beside our line: a sample of about this many
+# query/key pairs of the quantized-path simulation (about 10 s on 16 host
+# cores at d = 128), plus the full Q/K quantization.
+CPU_BASELINE_PAIRS = 1.2e8
+
+
+def cpu_sample_rows(w, target_pairs=CPU_BASELINE_PAIRS):
+    """Rows of the workload whose visible pairs add up to about target_pairs
+    (at least 64 rows, at most all of them)."""
+    total_rows = w.B * w.H * w.Lq
+    per_row = w.pairs() / total_rows
+    return int(min(total_rows, max(64, round(target_pairs / per_row))))
+
+
 def time_oracle_sample(w, q, k, v, n_rows, seed, qbr=128):
     """Oracle on a bounded sample: full Q/K quantization + n_rows query rows
     of the quantized-path simulation.  Returns (est_full_seconds, info)."""
@@ -480,7 +494,8 @@ def run_ours(args, w):
         torch.distributed.destroy_process_group()
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        est, info = time_oracle_sample(w, qn, kn, vn, args.cpu_rows, seed=0, qbr=qbr)
+        n_rows = args.cpu_rows if args.cpu_rows else cpu_sample_rows(w)
+        est, info = time_oracle_sample(w, qn, kn, vn, n_rows, seed=0, qbr=qbr)
         result["cpu_baseline"] = {
             "value": 4.0 * d * w.pairs() / est / 1e12, "unit": "TOPS",
             "cores": info["cores"], "kind": "oracle",
@@ -585,7 +600,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=10)
-    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--cpu-rows", type=int, default=0,
+                    help="query rows of the CPU-baseline sample (0: about "
+                         f"{CPU_BASELINE_PAIRS:.0e} query/key pairs' worth)")
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--q-block-rows", type=int, default=128, choices=[128, 64, 32, 1],

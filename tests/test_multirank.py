@@ -113,3 +113,15 @@ def test_secondary_ceilings_arithmetic():
     c8 = bench.secondary_ceilings(128, pairs, 0.1, 1.0, True, 148, 1965.0)
     assert c8["datasheet"]["t_roof_ms"] == pytest.approx(512 * pairs / 4.5e15 * 1e3)
     assert c8["exp2"]["max_roofline_frac"] == 1.0
+
+
+def test_cpu_baseline_sample_is_sized_by_pairs():
+    import bench
+    from bit_quantized_attention_mean_b200 import inputs
+    for w in inputs.WORKLOADS.values():
+        n = bench.cpu_sample_rows(w)
+        total = w.B * w.H * w.Lq
+        assert 64 <= n <= total or n == total
+        per_row = w.pairs() / total
+        if n < total:   # about the target, within one row
+            assert abs(n * per_row - bench.CPU_BASELINE_PAIRS) <= per_row
