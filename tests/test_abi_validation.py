@@ -48,6 +48,12 @@ def decode_varlen(H=8, Hkv=2, Lq=1, causal=0, qbr=1):
                                                                 S)
 
 
+def decode_paged(num_pages=16, max_blocks=8, table=A, lens=A, H=8, Hkv=2, Lq=1, qbr=1):
+    return sage.load_library().sage_attn_decode_prequant_paged(A, A, A, A, A, table, lens, A, 2,
+                                                               H, Hkv, Lq, num_pages, max_blocks,
+                                                               128, 1, qbr, N, 0, S)
+
+
 CASES = [
     ("quant_k: no keys", lambda: quant_k(Lk=0), INVALID),
     ("quant_k: d = 96", lambda: quant_k(d=96), UNSUPPORTED),
@@ -76,6 +82,13 @@ CASES = [
      UNSUPPORTED),
     ("decode: causal 3", lambda: decode_varlen(causal=3), INVALID),
     ("decode: block height 2", lambda: decode_varlen(qbr=2), INVALID),
+    ("paged: no pages", lambda: decode_paged(num_pages=0), INVALID),
+    ("paged: no block-table columns", lambda: decode_paged(max_blocks=0), INVALID),
+    ("paged: null block table", lambda: decode_paged(table=N), INVALID),
+    ("paged: null key counts", lambda: decode_paged(lens=N), INVALID),
+    ("paged: 16 heads x 9 queries > one tile", lambda: decode_paged(H=16, Hkv=1, Lq=9),
+     UNSUPPORTED),
+    ("paged: H % Hkv != 0", lambda: decode_paged(H=6, Hkv=4), INVALID),
 ]
 
 
