@@ -441,6 +441,50 @@ def test_sim_bottom_right_alignment_closed_form(Lq, Lk):
                                rtol=0, atol=1e-12)
 
 
+def _two_key_row(d=16):
+    """One query row, two keys: int8 scores S = (0, -1) with q_scale
+    fl32(1/3) and k_scale 1, so the base-2 scores are s = (0, -fl32(1/3))
+    and the row max is 0.  V rows: v0 = 0, v1 = 1 in every channel."""
+    q_i8 = np.zeros((1, 1, 1, d), np.int8); q_i8[..., 0] = 1
+    k_i8 = np.zeros((1, 1, 2, d), np.int8); k_i8[0, 0, 1, 0] = -1
+    q_scale = np.array([[[1 / 3]]], np.float32)
+    k_scale = np.ones((1, 1, 1), np.float32)
+    v = np.zeros((1, 1, 2, d), np.float16); v[0, 0, 1] = 1
+    s1 = -float(np.float32(1 / 3))
+    return q_i8, k_i8, q_scale, k_scale, v, s1
+
+
+def test_sim_rounds_p_to_fp16():
+    """P is held in fp16 (the FP16 P V step): with p1 = 2^s1 not an fp16
+    value, the output is p1h / (1 + p1h) with p1h = fp16(p1), computed here
+    with numpy's exp2 and float16 cast; the unrounded p1 moves it by ~1e-4."""
+    q_i8, k_i8, qs, ks, v, s1 = _two_key_row()
+    out = oracle.attn_quant_sim(q_i8, k_i8, qs, ks, v, False)
+    p1 = np.exp2(np.float64(s1))
+    p1h = float(np.float16(p1))
+    assert p1h != p1
+    np.testing.assert_allclose(out, np.full(out.shape, p1h / (1 + p1h)), rtol=0, atol=1e-15)
+    assert abs(p1h / (1 + p1h) - p1 / (1 + p1)) > 1e-6
+
+
+def test_fp8pv_sim_rounds_p_to_e4m3():
+    """FP8 path: P = e4m3(fl32(fl32(p) * 448)) / 448 (torch's float8_e4m3fn
+    conversion here), V = 1 is exact in E4M3 at scale 1/448, and the row sum
+    takes the unquantized p: out = P1 / (1 + p1)."""
+    import torch
+    q_i8, k_i8, qs, ks, v, s1 = _two_key_row()
+    v8t, vs = oracle.quant_v_fp8(v)
+    out = oracle.attn_fp8pv_sim(q_i8, k_i8, qs, ks, v8t, vs, False)
+    p1 = np.exp2(np.float64(s1))
+    x = np.float32(np.float32(p1) * np.float32(448.0))
+    p8 = float(torch.tensor([float(x)]).to(torch.float8_e4m3fn).float()[0]) / 448.0
+    assert p8 != p1
+    deq_v1 = float(torch.tensor([v8t[0, 0, 0, 1]], dtype=torch.uint8).view(
+        torch.float8_e4m3fn).float()[0]) * float(vs[0, 0, 0])
+    np.testing.assert_allclose(out, np.full(out.shape, p8 * deq_v1 / (1 + p1)), rtol=1e-15,
+                               atol=0)
+
+
 def test_sim_kv_block_permutation_invariance():
     q, k, v = inputs.make_custom(1, 1, 1, 64, 256, 64, seed=51)
     perm = np.array([2, 0, 3, 1])
