@@ -1,8 +1,13 @@
 """Benchmark of the 8-bit quantized attention forward pass on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload 1..5] [--q-block-rows 128|64|32|1] [--pv-accum f32|f16]
-                    [--decode]
+                    [--workload 1..5|all] [--q-block-rows 128|64|32|1]
+                    [--pv-accum f32|f16|fp8] [--decode]
+
+The default workload is the largest single-GPU configuration,
+longctx-causal-B1H16L32768d128-t4 (heavy-tailed inputs, per-token Q blocks:
+the Q granularity at which that workload meets the fp64 accuracy gate).
+``--workload all`` prints one line per workload 2..5 instead.
 
 A step is one pass of the whole hot path over the workload: K mean + Q/K
 quantization (sage_quant_qk) and the fused attention kernel
@@ -21,13 +26,17 @@ sums P V in fp16 as the SageAttention article states (sage_attn_fwd_ex /
 sage_attn_fwd_prequant_ex with SAGE_PV_ACCUM_F16).  ``roofline`` reports the attention
 kernel against the combined tensor roofline: QK at the INT8 peak and PV at the
 FP16 peak, t_roof = 2*d*pairs/P_int8 + 2*d*pairs/P_fp16, with P_fp16 the
-measured bf16 peak and P_int8 = 2 x P_fp16 (nominal dense ratio).
+measured bf16 peak and P_int8 measured in the same run (torch._int_mm at
+8192^3, best of 10); ``ceilings.nominal_int8`` repeats the fraction with
+P_int8 = 2 x P_fp16 (the datasheet ratio).
 
 Multi-GPU (torchrun, one process per GPU): every rank runs the same workload
 on its own GPU (the path shards by batch and head with no exchange, so this
 is weak scaling); value = all ranks' ops / the slowest rank's time.
 ``--impl reference`` times the CPU oracle (the only reference this path has)
-on a bounded row sample per step, on rank 0 only.
+on a bounded sample per step -- one (batch, head)'s Q/K quantization plus a
+few hundred of its query rows of the quantized-path simulation -- on rank 0
+only; its value is the sample's attention work over the sample's time.
 """
 from __future__ import annotations
 
@@ -49,7 +58,7 @@ sys.path.insert(0, ROOT)
 from bit_quantized_attention_mean_b200 import inputs  # noqa: E402
 
 METRIC = "quantized attention fwd TOPS at 1 B200 and % of INT8/FP16 tensor roofline"
-DEFAULT_WORKLOAD = 2
+DEFAULT_WORKLOAD = 5
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 INT8_OVER_FP16 = 2.0  # nominal dense ratio (4.5 / 2.25 PFLOP/s)
 # B200 datasheet dense peaks (TFLOP/s, per GPU) and the exp2 unit's rate
@@ -234,37 +243,69 @@ def weak_scaling_value(ops_per_rank, world, ms_per_step):
 
 # The one-off CPU baseline beside our line: a sample of about this many
 # query/key pairs of the quantized-path simulation (about 10 s on 16 host
-# cores at d = 128), plus the full Q/K quantization.
+# cores at d = 128), plus the quantization of the heads the rows fall in.
 CPU_BASELINE_PAIRS = 1.2e8
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or "unknown"
+
+
 def cpu_sample_rows(w, target_pairs=CPU_BASELINE_PAIRS):
-    """Rows of the workload whose visible pairs add up to about target_pairs
-    (at least 64 rows, at most all of them)."""
+    """Query rows whose visible pairs add up to about target_pairs (at least
+    64 rows, at most all of them)."""
     total_rows = w.B * w.H * w.Lq
     per_row = w.pairs() / total_rows
     return int(min(total_rows, max(64, round(target_pairs / per_row))))
 
 
-def time_oracle_sample(w, q, k, v, n_rows, seed, qbr=128):
-    """Oracle on a bounded sample: full Q/K quantization + n_rows query rows
-    of the quantized-path simulation.  Returns (est_full_seconds, info)."""
+def time_oracle_sample(w, q, k, v, n_rows, seed, qbr):
+    """The oracle on a bounded sample of the workload: n_rows random query
+    rows, spread over as few random (batch, head) pairs as hold them; for
+    each head, its Q and its kv head's K are quantized (the oracle's
+    quantization of that head alone, which is what it does for every head of
+    the full problem) and the sampled rows run through the quantized-path
+    simulation.  Returns (seconds, attention ops of the sampled rows, info)."""
     import oracle
     sm = float(np.float32(w.sm_scale))
-    t0 = time.perf_counter()
-    qk = oracle.quant_qk(q, k, sm, q_block_rows=qbr)
-    t_quant = time.perf_counter() - t0
     rng = np.random.default_rng(seed)
-    rows = np.sort(rng.choice(w.B * w.H * w.Lq, size=n_rows, replace=False)).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.attn_quant_sim(*qk[:4], v, w.causal, rows=rows, q_block_rows=qbr)
-    t_attn = time.perf_counter() - t0
-    i = rows % w.Lq
-    vis = np.minimum(w.Lk, np.maximum(0, i + (w.Lk - w.Lq) + 1)) if w.causal else np.full(n_rows, w.Lk)
-    sample_pairs = float(vis.sum())
-    est = t_quant + t_attn * (w.pairs() / sample_pairs)
-    return est, {"t_quant_s": t_quant, "t_attn_sample_s": t_attn, "rows": n_rows,
-                 "sample_pairs": sample_pairs, "cores": oracle.num_threads()}
+    heads = rng.permutation(w.B * w.H)
+    t_quant = t_attn = 0.0
+    pairs = 0
+    left = n_rows
+    used = 0
+    for bh in heads:
+        if left <= 0:
+            break
+        b, h = divmod(int(bh), w.H)
+        hk = h // (w.H // w.Hkv)
+        n = min(left, w.Lq)
+        rows = np.sort(rng.choice(w.Lq, size=n, replace=False)).astype(np.int64)
+        qh = np.ascontiguousarray(q[b:b + 1, h:h + 1])
+        kh = np.ascontiguousarray(k[b:b + 1, hk:hk + 1])
+        vh = np.ascontiguousarray(v[b:b + 1, hk:hk + 1])
+        t0 = time.perf_counter()
+        qk = oracle.quant_qk(qh, kh, sm, q_block_rows=qbr)
+        t1 = time.perf_counter()
+        oracle.attn_quant_sim(*qk[:4], vh, w.causal, rows=rows, q_block_rows=qbr)
+        t2 = time.perf_counter()
+        t_quant += t1 - t0
+        t_attn += t2 - t1
+        pairs += int(w.visible_keys(rows).sum())
+        left -= n
+        used += 1
+    ops = 4.0 * w.d * pairs
+    return t_quant + t_attn, ops, {"t_quant_s": t_quant, "t_attn_s": t_attn, "rows": n_rows,
+                                   "heads": used, "pairs": pairs,
+                                   "cores": oracle.num_threads()}
 
 
 def run_reference(args, w):
@@ -272,34 +313,60 @@ def run_reference(args, w):
     if rank != 0:
         return 0
     q, k, v = inputs.make_inputs(w)
-    ops = 4.0 * w.d * w.pairs()
+    qbr = args.q_block_rows
     rows = args.ref_rows
-    times = []
+    times, ops_l = [], []
     info = None
     for step in range(args.warmup + args.steps):
-        est, info = time_oracle_sample(w, q, k, v, rows, seed=step, qbr=args.q_block_rows)
+        t, ops, info = time_oracle_sample(w, q, k, v, rows, seed=step, qbr=qbr)
         if step >= args.warmup:
-            times.append(est)
+            times.append(t)
+            ops_l.append(ops)
     t = float(np.mean(times))
-    value = ops / t / 1e12
-    sample = (f"per step: oracle Q/K quantization of the full workload + quantized-path "
-              f"simulation of {rows} random query rows, time extrapolated to all "
-              f"{w.pairs()} query/key pairs")
+    value = float(np.sum(ops_l) / np.sum(times) / 1e12)
+    full_ms = 4.0 * w.d * w.pairs() / (value * 1e12) * 1e3
+    sample = (f"per step: one random (batch, head)'s Q/K quantization + quantized-path "
+              f"simulation of {rows} of its query rows (about "
+              f"{info['pairs'] / rows:.0f} visible keys each); value = those rows' "
+              f"attention ops / the step's time")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": t * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64 (int8 codes, int32 dot products)",
         "data": "synthetic (seeded numpy, fp16)",
-        "config": dict(w.describe(), q_block_rows=args.q_block_rows, pv_accum=args.pv_accum,
+        "config": dict(w.describe(), q_block_rows=qbr, pv_accum=args.pv_accum,
                        l2="n/a (CPU)"),
+        "extrapolated_full_workload_ms": full_ms,
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": info["cores"],
-                         "kind": "oracle", "sample": sample},
+                         "cpu_model": cpu_model(), "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def measure_int8_peak(dev, n=8192, reps=10):
+    """Dense INT8 GEMM rate of this GPU through cuBLAS (torch._int_mm, int8 x
+    int8 -> int32, n^3), best of `reps` CUDA-event timings, in TOPS."""
+    import torch
+    a = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev)
+    b = torch.randint(-127, 128, (n, n), dtype=torch.int8, device=dev).t().contiguous().t()
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize(dev)
+    best = float("inf")
+    for _ in range(reps):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize(dev)
+        best = min(best, e0.elapsed_time(e1))
+    del a, b
+    return 2.0 * n ** 3 / (best * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- ours
@@ -320,6 +387,7 @@ def run_ours(args, w):
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream(dev)
 
+    p_int8_meas = measure_int8_peak(dev) if args.int8_peak else None
     qn, kn, vn = inputs.make_inputs(w)
     sm = float(np.float32(w.sm_scale))
     q = torch.from_numpy(qn).to(dev)
@@ -333,8 +401,6 @@ def run_ours(args, w):
     q_scale = torch.empty((B, H, -(-Lq // qbr)), dtype=torch.float32, device=dev)
     k_scale = torch.empty((B, Hkv, -(-Lk // 64)), dtype=torch.float32, device=dev)
     k_mean = torch.empty((B, Hkv, d), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(1, sage.sage_quant_workspace_size(B, Hkv, Lk, d)), dtype=torch.uint8,
-                     device=dev)
     fp8 = args.pv_accum == "fp8"
     if fp8:
         v8t = torch.empty((B, Hkv, d, -(-Lk // 64) * 64), dtype=torch.uint8, device=dev)
@@ -348,11 +414,10 @@ def run_ours(args, w):
     def step():
         nonlocal launches
         if qbr == 128:
-            sage.sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, workspace=ws,
-                               stream=stream)
+            sage.sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, stream=stream)
         else:
             sage.sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm, qbr,
-                                      workspace=ws, stream=stream)
+                                      stream=stream)
         launches += sage.sage_last_launch_count()
         if fp8:   # V to E4M3 is part of the quantization step
             sage.sage_quant_v_fp8(v, v8t, v_scale, workspace=ws8, stream=stream)
@@ -411,11 +476,11 @@ def run_ours(args, w):
     e2e_steps = max(1, min(n, args.e2e_steps))
 
     def e2e_call():
-        if qbr == 128 and args.pv_accum == "f32":
-            sage.sage_attn_fwd_host(hq, hk, hv, hout, w.causal, sm, stream=stream)
+        if args.pv_accum == "f32":
+            sage.sage_attn_fwd_host_qblock(hq, hk, hv, hout, w.causal, sm, qbr, stream=stream)
             return
-        # finer Q blocks have no host-buffer entry point: the same copies,
-        # issued from here on the same stream around the device call
+        # the other P V variants have no host-buffer entry point: the same
+        # copies, issued from here on the same stream around the device call
         with torch.cuda.stream(stream):
             dq = hq.to(dev, non_blocking=True)
             dk = hk.to(dev, non_blocking=True)
@@ -449,15 +514,22 @@ def run_ours(args, w):
         value = weak_scaling_value(ops, world, ms_per_step)
         peaks = load_peaks()
         p16 = float(peaks["bf16_tflops"])
-        p8 = INT8_OVER_FP16 * p16
-        p_pv = p8 if fp8 else p16   # FP8 P V runs at the 8-bit rate
-        t_roof_ms = (2.0 * d * w.pairs() / (p8 * 1e12) + 2.0 * d * w.pairs() / (p_pv * 1e12)) * 1e3
+        p8_nominal = INT8_OVER_FP16 * p16
+        p8 = p_int8_meas if p_int8_meas else p8_nominal
+        p8_note = (f"P_int8 = {p8:.1f} TOPS measured in this run (torch._int_mm int8 8192^3, "
+                   f"best of 10)" if p_int8_meas else
+                   f"P_int8 = {INT8_OVER_FP16} x P_fp16 (nominal ratio)")
+
+        def roof_ms(pi8):
+            p_pv = pi8 if fp8 else p16   # FP8 P V runs at the 8-bit rate
+            return (2.0 * d * w.pairs() / (pi8 * 1e12) + 2.0 * d * w.pairs() / (p_pv * 1e12)) * 1e3
+        t_roof_ms = roof_ms(p8)
         peak_eff = ops / (t_roof_ms * 1e-3) / 1e12
         achieved = ops / (attn_avg_ms * 1e-3) / 1e12
         traffic = None
         if NCU_TRAFFIC.get("attn_sha") == attn_source_hash() and \
-                NCU_TRAFFIC.get("workload") == w.name and qbr == 128 and \
-                args.pv_accum == "f32":
+                NCU_TRAFFIC.get("workload") == w.name and \
+                NCU_TRAFFIC.get("q_block_rows", 128) == qbr and args.pv_accum == "f32":
             traffic = NCU_TRAFFIC.get("bytes_per_launch")
         quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d + 4 * B * H * -(-Lq // qbr)
         result = {
@@ -473,15 +545,18 @@ def run_ours(args, w):
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_eff,
                          "unit": "TFLOP/s", "frac": achieved / peak_eff, "traffic": traffic,
                          "kernel": "sage_attn_fwd_kernel",
-                         "peak_note": (f"combined roofline, QK at P_int8, PV at "
-                                       f"{'P_fp8 = P_int8' if fp8 else 'P_fp16'}: P_fp16 = {p16} "
-                                       f"TFLOP/s ({peaks.get('source')} bf16 burst), P_int8 = "
-                                       f"{INT8_OVER_FP16} x P_fp16 (nominal ratio)")},
+                         "peak_note": (f"combined roofline (of measured), QK at P_int8, PV "
+                                       f"at {'P_fp8 = P_int8' if fp8 else 'P_fp16'}: P_fp16 = "
+                                       f"{p16} TFLOP/s ({peaks.get('source')} bf16 burst), "
+                                       f"{p8_note}")},
             "kernel_ms": {"attention": attn_avg_ms, "quant": quant_avg_ms},
-            "ceilings": secondary_ceilings(
+            "ceilings": dict(secondary_ceilings(
                 d, w.pairs(), attn_avg_ms, t_roof_ms, fp8,
                 torch.cuda.get_device_properties(dev).multi_processor_count,
                 clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0),
+                nominal_int8={"frac": roof_ms(p8_nominal) / attn_avg_ms,
+                              "p_int8_tops": p8_nominal,
+                              "note": "same kernel time, P_int8 = 2 x measured bf16 peak"}),
             "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,
             "e2e": {"value": weak_scaling_value(ops, world, e2e_ms), "unit": "TOPS",
                     "h2d_bytes_per_step": int(qn.nbytes + kn.nbytes + vn.nbytes),
@@ -495,14 +570,15 @@ def run_ours(args, w):
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         n_rows = args.cpu_rows if args.cpu_rows else cpu_sample_rows(w)
-        est, info = time_oracle_sample(w, qn, kn, vn, n_rows, seed=0, qbr=qbr)
+        t, sample_ops, info = time_oracle_sample(w, qn, kn, vn, n_rows, seed=0, qbr=qbr)
         result["cpu_baseline"] = {
-            "value": 4.0 * d * w.pairs() / est / 1e12, "unit": "TOPS",
-            "cores": info["cores"], "kind": "oracle",
-            "sample": (f"oracle Q/K quantization of the full workload "
-                       f"({info['t_quant_s']:.2f} s) + quantized-path simulation of "
-                       f"{info['rows']} random query rows ({info['t_attn_sample_s']:.2f} s), "
-                       f"extrapolated to all query/key pairs")}
+            "value": sample_ops / t / 1e12, "unit": "TOPS",
+            "cores": info["cores"], "cpu_model": cpu_model(), "kind": "oracle",
+            "sample": (f"{info['rows']} random query rows in {info['heads']} random "
+                       f"(batch, head) pairs: the oracle's Q/K quantization of those heads "
+                       f"({info['t_quant_s']:.2f} s) + quantized-path simulation of the rows "
+                       f"({info['t_attn_s']:.2f} s, {info['pairs']} query/key pairs); value = "
+                       f"the rows' attention ops / that time")}
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
@@ -598,15 +674,19 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", type=int, default=DEFAULT_WORKLOAD, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--workload", default=str(DEFAULT_WORKLOAD),
+                    choices=[str(i) for i in sorted(inputs.WORKLOADS)] + ["all"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-rows", type=int, default=0,
                     help="query rows of the CPU-baseline sample (0: about "
                          f"{CPU_BASELINE_PAIRS:.0e} query/key pairs' worth)")
     ap.add_argument("--ref-rows", type=int, default=512)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--q-block-rows", type=int, default=128, choices=[128, 64, 32, 1],
-                    help="rows per Q quantization block (finer than the 128-row tile)")
+    ap.add_argument("--q-block-rows", type=int, default=None, choices=[128, 64, 32, 1],
+                    help="rows per Q quantization block (default: the workload's own, 128 "
+                         "except per-token for the long-context workload)")
+    ap.add_argument("--no-int8-peak", dest="int8_peak", action="store_false",
+                    help="skip the INT8 GEMM peak measurement (roofline then uses 2 x bf16)")
     ap.add_argument("--pv-accum", default="f32", choices=["f32", "f16", "fp8"],
                     help="P V variant: fp16 P/V with fp32 sums (default), fp16 sums as the "
                          "article states, or P and V in FP8 E4M3 (SageAttention2)")
@@ -618,10 +698,15 @@ def main():
     if args.decode:
         return run_decode_bench(args) if args.impl == "ours" else print(json.dumps(
             {"impl": "reference", "unavailable": "the decode timing has no CPU reference arm"}))
-    w = inputs.WORKLOADS[args.workload]
-    if args.impl == "reference":
-        return run_reference(args, w)
-    return run_ours(args, w)
+    ids = [2, 3, 4, 5] if args.workload == "all" else [int(args.workload)]
+    qbr_arg = args.q_block_rows
+    for i in ids:
+        w = inputs.WORKLOADS[i]
+        args.q_block_rows = qbr_arg if qbr_arg is not None else w.q_block_rows
+        rc = run_reference(args, w) if args.impl == "reference" else run_ours(args, w)
+        if rc:
+            return rc
+    return 0
 
 
 if __name__ == "__main__":

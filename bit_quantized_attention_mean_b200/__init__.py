@@ -13,8 +13,8 @@ Exported names mirror the C ABI:
     sage_attn_decode, sage_attn_decode_prequant, sage_attn_decode_workspace_size,
     sage_quant_v_fp8, sage_quant_v_fp8_workspace_size, sage_attn_fwd_prequant_fp8pv,
     sage_quant_qk_varlen, sage_attn_fwd_prequant_varlen, sage_attn_fwd_varlen,
-    sage_quant_k,
-    sage_quant_workspace_size, sage_attn_workspace_size,
+    sage_quant_k, sage_attn_fwd_host, sage_attn_fwd_host_qblock, sage_attn_fwd_noalloc,
+    sage_workspace_size,
     sage_check_device_status, sage_status_string, sage_last_launch_count
 plus conveniences that allocate outputs: ``quant_qk``, ``attention``,
 ``attention_varlen`` and ``decode``.
@@ -28,6 +28,7 @@ from ._lib import (  # noqa: F401
     load_library,
     sage_attn_fwd,
     sage_attn_fwd_host,
+    sage_attn_fwd_host_qblock,
     sage_attn_fwd_noalloc,
     NOALLOC_SCRATCH_BYTES,
     sage_attn_fwd_prequant,
@@ -37,13 +38,12 @@ from ._lib import (  # noqa: F401
     sage_attn_fwd_prequant_ex,
     SAGE_PV_ACCUM_F16,
     PV_ACCUM,
-    sage_attn_workspace_size,
+    sage_workspace_size,
     sage_check_device_status,
     sage_debug_wait_timeout,
     sage_last_launch_count,
     sage_quant_qk,
     sage_quant_qk_qblock,
-    sage_quant_workspace_size,
     Q_BLOCK_ROWS,
     sage_status_string,
     quant_qk,

@@ -18,11 +18,11 @@ _lib = None
 # Every symbol include/sage.h declares.
 SYMBOLS = (
     "sage_quant_qk",
-    "sage_quant_workspace_size",
+    "sage_workspace_size",
     "sage_attn_fwd_prequant",
     "sage_attn_fwd",
     "sage_attn_fwd_host",
-    "sage_attn_workspace_size",
+    "sage_attn_fwd_host_qblock",
     "sage_check_device_status",
     "sage_status_string",
     "sage_last_launch_count",
@@ -78,18 +78,18 @@ def load_library():
                 "`python -m bit_quantized_attention_mean_b200.build` (no fallback exists)")
         lib = ctypes.CDLL(_LIB_PATH)
         P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
-        lib.sage_quant_qk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, Z, P]
+        lib.sage_quant_qk.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P]
         lib.sage_quant_qk.restype = I
-        lib.sage_quant_workspace_size.argtypes = [I, I, I, I]
-        lib.sage_quant_workspace_size.restype = Z
         lib.sage_attn_fwd_prequant.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, P]
         lib.sage_attn_fwd_prequant.restype = I
         lib.sage_attn_fwd.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
         lib.sage_attn_fwd.restype = I
         lib.sage_attn_fwd_host.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, P]
         lib.sage_attn_fwd_host.restype = I
-        lib.sage_attn_workspace_size.argtypes = [I, I, I, I, I, I]
-        lib.sage_attn_workspace_size.restype = Z
+        lib.sage_attn_fwd_host_qblock.argtypes = [P, P, P, P, I, I, I, I, I, I, I, F, I, P]
+        lib.sage_attn_fwd_host_qblock.restype = I
+        lib.sage_workspace_size.argtypes = [I, I, I, I, I, I]
+        lib.sage_workspace_size.restype = Z
         lib.sage_check_device_status.argtypes = [P]
         lib.sage_check_device_status.restype = I
         lib.sage_status_string.argtypes = [I]
@@ -98,8 +98,7 @@ def load_library():
         lib.sage_attn_fwd_noalloc.restype = I
         lib.sage_debug_wait_timeout.argtypes = [I, P]
         lib.sage_debug_wait_timeout.restype = I
-        lib.sage_quant_qk_qblock.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P, Z,
-                                             P]
+        lib.sage_quant_qk_qblock.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I, F, I, P]
         lib.sage_quant_qk_qblock.restype = I
         lib.sage_attn_fwd_prequant_qblock.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, I,
                                                       P]
@@ -130,14 +129,14 @@ def load_library():
                                                         I, I, I, P, Z, P]
         lib.sage_attn_decode_prequant_paged.restype = I
         lib.sage_quant_qk_varlen.argtypes = [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, F, I,
-                                             P, Z, P]
+                                             P]
         lib.sage_quant_qk_varlen.restype = I
         lib.sage_attn_fwd_prequant_varlen.argtypes = [P, P, P, P, P, P, P, P, I, I, I, I, I, I,
                                                       I, I, U, P]
         lib.sage_attn_fwd_prequant_varlen.restype = I
         lib.sage_attn_fwd_varlen.argtypes = [P, P, P, P, P, P, I, I, I, I, I, I, I, F, I, U, P]
         lib.sage_attn_fwd_varlen.restype = I
-        lib.sage_quant_k.argtypes = [P, P, P, P, I, I, I, I, P, Z, P]
+        lib.sage_quant_k.argtypes = [P, P, P, P, I, I, I, I, P]
         lib.sage_quant_k.restype = I
         lib.sage_last_launch_count.argtypes = []
         lib.sage_last_launch_count.restype = I
@@ -190,12 +189,9 @@ def sage_last_launch_count() -> int:
     return load_library().sage_last_launch_count()
 
 
-def sage_quant_workspace_size(B, Hkv, Lk, d) -> int:
-    return load_library().sage_quant_workspace_size(B, Hkv, Lk, d)
-
-
-def sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
-    return load_library().sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d)
+def sage_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
+    """Bytes of device scratch sage_attn_fwd allocates for this shape."""
+    return load_library().sage_workspace_size(B, H, Hkv, Lq, Lk, d)
 
 
 def _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, q_block_rows):
@@ -224,22 +220,21 @@ def _check_qbr(q_block_rows):
         raise ValueError(f"q_block_rows must be one of {Q_BLOCK_ROWS}, got {q_block_rows}")
 
 
-def sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale,
-                  workspace=None, stream=None):
+def sage_quant_qk(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, stream=None):
     """Smooth K and quantize Q/K per block into the given output tensors."""
     args = _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, 128)
-    _check(load_library().sage_quant_qk(*args, float(sm_scale), *_workspace(workspace),
-                                        _stream(stream)), "sage_quant_qk")
+    _check(load_library().sage_quant_qk(*args, float(sm_scale), _stream(stream)),
+           "sage_quant_qk")
 
 
 def sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, sm_scale, q_block_rows,
-                         workspace=None, stream=None):
+                         stream=None):
     """sage_quant_qk with Q blocks of q_block_rows rows (128, 64, 32 or 1);
     q_scale has shape [B, H, ceil(Lq / q_block_rows)]."""
     _check_qbr(q_block_rows)
     args = _quant_args(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, q_block_rows)
     _check(load_library().sage_quant_qk_qblock(*args, float(sm_scale), int(q_block_rows),
-                                               *_workspace(workspace), _stream(stream)),
+                                               _stream(stream)),
            "sage_quant_qk_qblock")
 
 
@@ -345,7 +340,7 @@ def _seqlens(t, name, B):
 
 
 def sage_quant_qk_varlen(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, seqlens_q, seqlens_k,
-                         sm_scale, q_block_rows=128, workspace=None, stream=None):
+                         sm_scale, q_block_rows=128, stream=None):
     """sage_quant_qk_qblock on a padded batch: entry b quantizes its first
     seqlens_q[b] Q rows and smooths/quantizes its first seqlens_k[b] keys
     (int32 CUDA tensors [B], or None for all rows / all keys)."""
@@ -354,7 +349,7 @@ def sage_quant_qk_varlen(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, seqlens_q, 
     B = q.shape[0]
     _check(load_library().sage_quant_qk_varlen(
         *args[:7], _seqlens(seqlens_q, "seqlens_q", B), _seqlens(seqlens_k, "seqlens_k", B),
-        *args[7:], float(sm_scale), int(q_block_rows), *_workspace(workspace), _stream(stream)),
+        *args[7:], float(sm_scale), int(q_block_rows), _stream(stream)),
         "sage_quant_qk_varlen")
 
 
@@ -394,7 +389,7 @@ def sage_attn_fwd_varlen(q, k, v, out, seqlens_q, seqlens_k, causal, sm_scale, q
         _stream(stream)), "sage_attn_fwd_varlen")
 
 
-def sage_quant_k(k, k_i8, k_scale, k_mean, workspace=None, stream=None):
+def sage_quant_k(k, k_i8, k_scale, k_mean, stream=None):
     """Smooth K and quantize it in 64-row blocks (the K half of
     sage_quant_qk) into the given output tensors."""
     import torch
@@ -403,7 +398,7 @@ def sage_quant_k(k, k_i8, k_scale, k_mean, workspace=None, stream=None):
         _dev(k, torch.float16, "k"), _dev(k_i8, torch.int8, "k_i8", k.shape),
         _dev(k_scale, torch.float32, "k_scale", (B, Hkv, -(-Lk // 64))),
         _dev(k_mean, torch.float32, "k_mean", (B, Hkv, d)), B, Hkv, Lk, d,
-        *_workspace(workspace), _stream(stream)), "sage_quant_k")
+        _stream(stream)), "sage_quant_k")
 
 
 def sage_attn_decode_workspace_size(B, H, Hkv, Lq, Lk, d) -> int:
@@ -537,7 +532,7 @@ def sage_attn_fwd_noalloc(q, k, v, out, causal, sm_scale, stream=None):
     library).  The library's scratch is one fixed 64 MiB device array shared by
     all calls: order the calls on one stream, make the first call on a device
     before any stream capture, and keep problems within the array
-    (sage_attn_workspace_size(...) <= 64 MiB), else SageError is raised."""
+    (sage_workspace_size(...) <= 64 MiB), else SageError is raised."""
     import torch
     lib = load_library()
     B, H, Hkv, Lq, Lk, d = _dims(q, k)
@@ -546,7 +541,7 @@ def sage_attn_fwd_noalloc(q, k, v, out, causal, sm_scale, stream=None):
         _dev(v, torch.float16, "v", k.shape), _dev(out, torch.float16, "out", q.shape),
         B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream))
     if status != 0:
-        need = lib.sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d)
+        need = lib.sage_workspace_size(B, H, Hkv, Lq, Lk, d)
         if status == 1 and need > NOALLOC_SCRATCH_BYTES:
             raise SageError(status, f"sage_attn_fwd_noalloc (needs {need} bytes of scratch, "
                                     f"the fixed array holds {NOALLOC_SCRATCH_BYTES})")
@@ -555,7 +550,13 @@ def sage_attn_fwd_noalloc(q, k, v, out, causal, sm_scale, stream=None):
 
 def sage_attn_fwd_host(q, k, v, out, causal, sm_scale, stream=None):
     """Whole forward pass on HOST fp16 tensors (pinned for async copies)."""
+    sage_attn_fwd_host_qblock(q, k, v, out, causal, sm_scale, 128, stream)
+
+
+def sage_attn_fwd_host_qblock(q, k, v, out, causal, sm_scale, q_block_rows, stream=None):
+    """sage_attn_fwd_host with Q quantized in blocks of q_block_rows rows."""
     import torch
+    _check_qbr(q_block_rows)
     lib = load_library()
     for name, t in (("q", q), ("k", k), ("v", v), ("out", out)):
         if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.float16 \
@@ -564,11 +565,11 @@ def sage_attn_fwd_host(q, k, v, out, causal, sm_scale, stream=None):
     B, H, Hkv, Lq, Lk, d = _dims(q, k)
     if tuple(v.shape) != tuple(k.shape) or tuple(out.shape) != tuple(q.shape):
         raise ValueError("v must match k and out must match q")
-    _check(lib.sage_attn_fwd_host(
+    _check(lib.sage_attn_fwd_host_qblock(
         ctypes.c_void_p(q.data_ptr()), ctypes.c_void_p(k.data_ptr()),
         ctypes.c_void_p(v.data_ptr()), ctypes.c_void_p(out.data_ptr()),
-        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), _stream(stream)),
-        "sage_attn_fwd_host")
+        B, H, Hkv, Lq, Lk, d, 1 if causal else 0, float(sm_scale), int(q_block_rows),
+        _stream(stream)), "sage_attn_fwd_host_qblock")
 
 
 def sage_debug_wait_timeout(limit_ms, stream=None):

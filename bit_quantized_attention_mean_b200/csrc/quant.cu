@@ -313,8 +313,6 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
 
 // ------------------------------------------------------------- launcher
 
-size_t quant_workspace_bytes(int, int, int, int) { return 0; }
-
 template <int D, int QBR>
 static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* launches) {
   const int BH = a.B * a.H, BHkv = a.B * a.Hkv;
@@ -327,7 +325,9 @@ static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* laun
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)
     cl = 16;
   const int kb_per_cta = (nkb + cl - 1) / cl;
-  // a CTA sums at most kb_per_cta * 64 rows; each thread at most 1/RPP of them
+  // a CTA sums at most kb_per_cta * 64 rows and each thread at most 1/RPP of
+  // them, at most 2^13 exact double sums; the entry points refuse Lk above
+  // SAGE_MAX_LK (2^20), which keeps this bound for every cluster width and d
   if ((long long)kb_per_cta * SAGE_K_BLOCK_ROWS / (kQuantThreads / (D / 8)) > 8192)
     return cudaErrorInvalidValue;
   const long long n_k_ctas = (long long)BHkv * cl;

@@ -13,34 +13,11 @@ namespace {
 
 thread_local int g_last_launches = 0;
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-sage_status check_shape(int B, int H, int Hkv, int Lq, int Lk, int d) {
-  if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1) return SAGE_ERR_INVALID_ARG;
-  if (H % Hkv != 0) return SAGE_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
-  // every element offset and grid size must fit the kernels' index types
-  const long long qn = (long long)B * H * Lq, kn = (long long)B * Hkv * Lk;
-  if (qn * d > (1LL << 40) || kn * d > (1LL << 40)) return SAGE_ERR_INVALID_ARG;
-  if (qn / 128 + 1 > 0x7fffffffLL || kn / 64 + 1 > 0x7fffffffLL) return SAGE_ERR_INVALID_ARG;
-  return SAGE_OK;
-}
-
-sage_status check_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
-  int major = 0, minor = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return SAGE_ERR_CUDA;
-  if (major != 10 || minor != 0) return SAGE_ERR_UNSUPPORTED;  // built for sm_100a only
-  return SAGE_OK;
-}
-
-float fold_constant(float sm_scale) {
-  // c = fl32(double(sm_scale) * log2(e)); folded into the Q scales
-  return (float)((double)sm_scale * 1.4426950408889634074);
-}
+using sage::aligned16;
+using sage::check_device;
+using sage::check_quant_len;
+using sage::check_shape;
+using sage::fold_constant;
 
 size_t round_up(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -71,7 +48,7 @@ cudaStream_t* side_streams(int dev) {
 }
 
 struct AttnWorkspace {
-  size_t q_i8, k_i8, q_scale, k_scale, k_mean, part, total;
+  size_t q_i8, k_i8, q_scale, k_scale, k_mean, total;
 };
 
 AttnWorkspace attn_workspace_layout(int B, int H, int Hkv, int Lq, int Lk, int d, int qbr) {
@@ -83,12 +60,15 @@ AttnWorkspace attn_workspace_layout(int B, int H, int Hkv, int Lq, int Lk, int d
   w.q_scale = off; off += round_up((size_t)B * H * nqb * 4);
   w.k_scale = off; off += round_up((size_t)B * Hkv * nkb * 4);
   w.k_mean = off;  off += round_up((size_t)B * Hkv * d * 4);
-  w.part = off;    off += round_up(sage::quant_workspace_bytes(B, Hkv, Lk, d));
   w.total = off;
   return w;
 }
 
 }  // namespace
+
+namespace sage {
+void set_last_launch_count(int n) { g_last_launches = n; }
+}  // namespace sage
 
 extern "C" {
 
@@ -105,61 +85,49 @@ const char* sage_status_string(sage_status s) {
 
 int sage_last_launch_count(void) { return g_last_launches; }
 
-size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d) {
-  if (B < 1 || Hkv < 1 || Lk < 1 || (d != 64 && d != 128)) return 0;
-  return sage::quant_workspace_bytes(B, Hkv, Lk, d);
-}
-
-size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
+size_t sage_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d) {
   if (check_shape(B, H, Hkv, Lq, Lk, d) != SAGE_OK) return 0;
   return attn_workspace_layout(B, H, Hkv, Lq, Lk, d, SAGE_Q_BLOCK).total;
 }
 
 sage_status sage_quant_qk(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8, float* q_scale,
                           float* k_scale, float* k_mean, int B, int H, int Hkv, int Lq, int Lk,
-                          int d, float sm_scale, void* workspace, size_t workspace_bytes,
-                          void* stream) {
+                          int d, float sm_scale, void* stream) {
   return sage_quant_qk_qblock(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, B, H, Hkv, Lq, Lk, d,
-                              sm_scale, SAGE_Q_BLOCK, workspace, workspace_bytes, stream);
+                              sm_scale, SAGE_Q_BLOCK, stream);
 }
 
 sage_status sage_quant_qk_qblock(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8,
                                  float* q_scale, float* k_scale, float* k_mean, int B, int H,
                                  int Hkv, int Lq, int Lk, int d, float sm_scale, int q_block_rows,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+                                 void* stream) {
   return sage_quant_qk_varlen(q, k, q_i8, k_i8, q_scale, k_scale, k_mean, nullptr, nullptr, B, H,
-                              Hkv, Lq, Lk, d, sm_scale, q_block_rows, workspace, workspace_bytes,
-                              stream);
+                              Hkv, Lq, Lk, d, sm_scale, q_block_rows, stream);
 }
 
 sage_status sage_quant_qk_varlen(const void* q, const void* k, int8_t* q_i8, int8_t* k_i8,
                                  float* q_scale, float* k_scale, float* k_mean,
                                  const int* seqlens_q, const int* seqlens_k, int B, int H,
                                  int Hkv, int Lq, int Lk, int d, float sm_scale, int q_block_rows,
-                                 void* workspace, size_t workspace_bytes, void* stream) {
+                                 void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if ((st = check_quant_len(Lk)) != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !q_i8 || !k_i8 || !q_scale || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8) ||
       !aligned16(q_scale) || !aligned16(k_scale) || !aligned16(k_mean))
     return SAGE_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  const size_t need = sage::quant_workspace_bytes(B, Hkv, Lk, d);
-  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
   if ((st = check_device()) != SAGE_OK) return st;
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void* ws = workspace;
-  const bool own = !ws && need > 0;
-  if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
   sage::QuantArgs a{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
-                    q_scale, k_scale, k_mean, ws, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale),
+                    q_scale, k_scale, k_mean, B, H, Hkv, Lq, Lk, d, fold_constant(sm_scale),
                     q_block_rows, seqlens_q, seqlens_k};
   int launches = 0;
   cudaError_t e = sage::launch_quant(a, s, &launches);
-  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
   g_last_launches = launches;
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
@@ -244,6 +212,7 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if ((st = check_quant_len(Lk)) != SAGE_OK) return st;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!valid_flags(flags)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
@@ -269,7 +238,7 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
   float* k_scale = reinterpret_cast<float*>(ws + w.k_scale);
   float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
   sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
-                     q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
+                     q_scale, k_scale, k_mean, B, H, Hkv, Lq, Lk, d,
                      fold_constant(sm_scale), q_block_rows, seqlens_q, seqlens_k};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
@@ -297,27 +266,21 @@ sage_status sage_attn_fwd_varlen(const void* q, const void* k, const void* v, vo
 }
 
 sage_status sage_quant_k(const void* k, int8_t* k_i8, float* k_scale, float* k_mean, int B,
-                         int Hkv, int Lk, int d, void* workspace, size_t workspace_bytes,
-                         void* stream) {
+                         int Hkv, int Lk, int d, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, Hkv, Hkv, 1, Lk, d);
   if (st != SAGE_OK) return st;
+  if ((st = check_quant_len(Lk)) != SAGE_OK) return st;
   if (!k || !k_i8 || !k_scale || !k_mean) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(k_i8) || !aligned16(k_scale) || !aligned16(k_mean))
     return SAGE_ERR_INVALID_ARG;
-  const size_t need = sage::quant_workspace_bytes(B, Hkv, Lk, d);
-  if (workspace && (workspace_bytes < need || !aligned16(workspace))) return SAGE_ERR_INVALID_ARG;
   if ((st = check_device()) != SAGE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  void* ws = workspace;
-  const bool own = !ws && need > 0;
-  if (own && cudaMallocAsync(&ws, need, s) != cudaSuccess) return SAGE_ERR_CUDA;
   sage::QuantArgs a{nullptr, static_cast<const __half*>(k), nullptr, k_i8, nullptr, k_scale,
-                    k_mean, ws, B, Hkv, Hkv, 1, Lk, d, 1.f, SAGE_Q_BLOCK};
+                    k_mean, B, Hkv, Hkv, 1, Lk, d, 1.f, SAGE_Q_BLOCK};
   a.skip_q = true;
   int launches = 0;
   cudaError_t e = sage::launch_quant(a, s, &launches);
-  if (own && cudaFreeAsync(ws, s) != cudaSuccess && e == cudaSuccess) e = cudaErrorUnknown;
   g_last_launches = launches;
   return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA;
 }
@@ -426,6 +389,7 @@ sage_status sage_attn_decode(const void* q, const void* k, const void* v, void* 
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if ((st = check_quant_len(Lk)) != SAGE_OK) return st;
   if ((long long)(H / Hkv) * Lq > 128) return SAGE_ERR_UNSUPPORTED;
   if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q || !k || !v || !out) return SAGE_ERR_INVALID_ARG;
@@ -447,7 +411,7 @@ sage_status sage_attn_decode(const void* q, const void* k, const void* v, void* 
   float* k_scale = reinterpret_cast<float*>(ws + w.k_scale);
   float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
   sage::QuantArgs qa{static_cast<const __half*>(q), static_cast<const __half*>(k), q_i8, k_i8,
-                     q_scale, k_scale, k_mean, ws + w.part, B, H, Hkv, Lq, Lk, d,
+                     q_scale, k_scale, k_mean, B, H, Hkv, Lq, Lk, d,
                      fold_constant(sm_scale), q_block_rows};
   int launches = 0;
   cudaError_t e = sage::launch_quant(qa, s, &launches);
@@ -521,9 +485,19 @@ sage_status sage_attn_fwd_prequant_fp8pv(const int8_t* q_i8, const int8_t* k_i8,
 sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const void* v_host,
                                void* out_host, int B, int H, int Hkv, int Lq, int Lk, int d,
                                int causal, float sm_scale, void* stream) {
+  return sage_attn_fwd_host_qblock(q_host, k_host, v_host, out_host, B, H, Hkv, Lq, Lk, d, causal,
+                                   sm_scale, SAGE_Q_BLOCK, stream);
+}
+
+sage_status sage_attn_fwd_host_qblock(const void* q_host, const void* k_host,
+                                      const void* v_host, void* out_host, int B, int H, int Hkv,
+                                      int Lq, int Lk, int d, int causal, float sm_scale,
+                                      int q_block_rows, void* stream) {
   g_last_launches = 0;
   sage_status st = check_shape(B, H, Hkv, Lq, Lk, d);
   if (st != SAGE_OK) return st;
+  if ((st = check_quant_len(Lk)) != SAGE_OK) return st;
+  if (!sage::valid_q_block_rows(q_block_rows)) return SAGE_ERR_INVALID_ARG;
   if (!q_host || !k_host || !v_host || !out_host) return SAGE_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return SAGE_ERR_INVALID_ARG;
   if (!(sm_scale > 0.f) || !std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
@@ -547,7 +521,7 @@ sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const voi
   const int per = (groups + nchunk - 1) / nchunk;
   const size_t qh = (size_t)Lq * d * 2, kh = (size_t)Lk * d * 2;  // bytes per head
   const size_t qb = (size_t)B * H * qh, kb = (size_t)B * Hkv * kh;
-  const AttnWorkspace w = attn_workspace_layout(1, per * G, per, Lq, Lk, d, SAGE_Q_BLOCK);
+  const AttnWorkspace w = attn_workspace_layout(1, per * G, per, Lq, Lk, d, q_block_rows);
   const size_t total = round_up(qb) * 2 + round_up(kb) * 2 + w.total;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   char* buf = nullptr;
@@ -602,12 +576,12 @@ sage_status sage_attn_fwd_host(const void* q_host, const void* k_host, const voi
       float* k_mean = reinterpret_cast<float*>(ws + w.k_mean);
       sage::QuantArgs qa{reinterpret_cast<const __half*>(dq + qo),
                          reinterpret_cast<const __half*>(dk + ko), q_i8, k_i8, q_scale, k_scale,
-                         k_mean, ws + w.part, 1, n * G, n, Lq, Lk, d, c, SAGE_Q_BLOCK};
+                         k_mean, 1, n * G, n, Lq, Lk, d, c, q_block_rows};
       e = sage::launch_quant(qa, comp, &launches);
       if (e == cudaSuccess) {
         sage::AttnArgs aa{q_i8, k_i8, q_scale, k_scale, reinterpret_cast<const __half*>(dv + ko),
                           reinterpret_cast<__half*>(dout + qo), 1, n * G, n, Lq, Lk, d,
-                          causal == 1, SAGE_Q_BLOCK, false};
+                          causal == 1, q_block_rows, false};
         e = sage::launch_attn(aa, comp, &launches);
       }
     }

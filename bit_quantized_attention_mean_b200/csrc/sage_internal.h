@@ -8,10 +8,55 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "../../include/sage.h"
+
 #define SAGE_Q_BLOCK_ROWS 128
 #define SAGE_K_BLOCK_ROWS 64
 
 namespace sage {
+
+// ------------------------------------------------ host-side argument checks
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape rules shared by every entry point: positive sizes, H a multiple of
+// Hkv, d in {64, 128}, and element offsets / grid sizes that fit the
+// kernels' index types.
+inline sage_status check_shape(int B, int H, int Hkv, int Lq, int Lk, int d) {
+  if (B < 1 || H < 1 || Hkv < 1 || Lq < 1 || Lk < 1) return SAGE_ERR_INVALID_ARG;
+  if (H % Hkv != 0) return SAGE_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SAGE_ERR_UNSUPPORTED;
+  const long long qn = (long long)B * H * Lq, kn = (long long)B * Hkv * Lk;
+  if (qn * d > (1LL << 40) || kn * d > (1LL << 40)) return SAGE_ERR_INVALID_ARG;
+  if (qn / 128 + 1 > 0x7fffffffLL || kn / 64 + 1 > 0x7fffffffLL) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+// The quantization kernel's exact K column sums hold at most SAGE_MAX_LK keys
+// per (batch, kv head); every call that quantizes K checks this first.
+inline sage_status check_quant_len(int Lk) {
+  return Lk > SAGE_MAX_LK ? SAGE_ERR_UNSUPPORTED : SAGE_OK;
+}
+
+// sm_100 device current (the library is built for sm_100a only).
+inline sage_status check_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  if (major != 10 || minor != 0) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+// c = fl32(double(sm_scale) * log2(e)), folded into the Q scales.
+inline float fold_constant(float sm_scale) {
+  return (float)((double)sm_scale * 1.4426950408889634074);
+}
+
+// Records what sage_last_launch_count() reports for this thread.
+void set_last_launch_count(int n);
 
 struct QuantArgs {
   const __half* q;
@@ -21,7 +66,6 @@ struct QuantArgs {
   float* q_scale;
   float* k_scale;
   float* k_mean;
-  void* workspace;  // quant_workspace_bytes() of scratch (int64 partial sums)
   int B, H, Hkv, Lq, Lk, d;
   float c;          // fl32(double(sm_scale) * log2(e)), folded into q_scale
   int q_block_rows; // rows per Q quantization block: 128, 64, 32 or 1
@@ -90,8 +134,6 @@ struct DecodePlan {
 DecodePlan decode_plan(int B, int H, int Hkv, int Lq, int Lk, int d);
 cudaError_t launch_decode(const DecodeArgs& a, const DecodePlan& p, cudaStream_t st,
                           int* launches);
-
-size_t quant_workspace_bytes(int B, int Hkv, int Lk, int d);
 
 // Each launcher adds the number of kernels it launched to *launches and
 // returns the first CUDA error (cudaSuccess when every launch was accepted).

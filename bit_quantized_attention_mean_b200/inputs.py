@@ -41,6 +41,9 @@ class Workload:
     outlier_magnitude: float = 0.0
     v_scale: float = 1.0
     student_t: bool = False
+    # Q quantization block rows this workload is run with: the 128-row tile,
+    # or one row per block where 128-row blocks miss the fp64 accuracy gate
+    q_block_rows: int = 128
 
     @property
     def Lq(self) -> int:
@@ -65,6 +68,13 @@ class Workload:
             "Lk": self.Lk, "d": self.d, "causal": self.causal,
         }
 
+    def visible_keys(self, rows: "np.ndarray") -> "np.ndarray":
+        """Keys visible to each of the given within-head row indices."""
+        rows = np.asarray(rows, dtype=np.int64)
+        if not self.causal:
+            return np.full(rows.shape, self.Lk, dtype=np.int64)
+        return np.clip(rows + (self.Lk - self.Lq) + 1, 0, self.Lk)
+
 
 def visible_pairs(B: int, H: int, Lq: int, Lk: int, causal: bool) -> int:
     """Count of (i, j) with key j visible to query i (bottom-right causal)."""
@@ -86,7 +96,7 @@ WORKLOADS = {
                 v_scale=4.0),
     4: Workload(4, "gqa-causal-B4H32Hkv8L8192d128", 4, 32, 8, 8192, 128, True, 2.0),
     5: Workload(5, "longctx-causal-B1H16L32768d128-t4", 1, 16, 16, 32768, 128, True, 3.0,
-                student_t=True),
+                student_t=True, q_block_rows=1),
 }
 
 

@@ -31,6 +31,10 @@
  *     or allocation returns SAGE_ERR_CUDA.  Errors inside a kernel (a bounded
  *     wait that gave up) are recorded in a device status word, read by
  *     sage_check_device_status().
+ *   - Every call that smooths and quantizes K (sage_quant_qk*, sage_quant_k,
+ *     sage_attn_fwd, its _qblock/_ex/_varlen/_host/_noalloc forms and
+ *     sage_attn_decode) accepts Lk <= SAGE_MAX_LK and returns
+ *     SAGE_ERR_UNSUPPORTED for a longer K, before any launch.
  *   - Inputs must be finite; NaN/Inf inputs give unspecified outputs.
  */
 #ifndef SAGE_B200_H
@@ -61,6 +65,9 @@ typedef enum {
 #define SAGE_Q_BLOCK 128
 #define SAGE_K_BLOCK 64
 
+/* Longest K (keys per (batch, kv head)) the quantizing calls accept. */
+#define SAGE_MAX_LK (1 << 20)
+
 /* Flags of the _ex entry points. */
 #define SAGE_PV_ACCUM_F16 1u  /* accumulate P V in fp16 (the article's choice) */
 #define SAGE_PV_FP8 2u        /* P and V in FP8 E4M3, fp32 sums (SageAttention2) */
@@ -76,12 +83,11 @@ typedef enum {
  *                                          c = fl32(double(sm_scale)*log2(e))
  *   k_scale  fp32 [B, Hkv, ceil(Lk/64)]    (out) fl32(amax/127)
  *   k_mean   fp32 [B, Hkv, d]              (out) mean of K over all Lk tokens
- *   workspace, workspace_bytes: device scratch of at least
- *            sage_quant_workspace_size(B, Hkv, Lk, d) bytes, or NULL/0 to let
- *            the call allocate it with cudaMallocAsync on `stream`.  The
- *            current kernels need none (the size is 0; the K mean is reduced
- *            in on-chip distributed shared memory), so NULL/0 is always fine.
  *
+ * Needs no scratch memory: the K mean is reduced exactly in on-chip
+ * distributed shared memory.  Lk may be at most SAGE_MAX_LK (2^20) keys: a
+ * longer K returns SAGE_ERR_UNSUPPORTED before anything is launched (the
+ * exact per-thread column sums of the K mean are sized for it).
  * Per block: a = max|x|, r = fl32(127/a), q = clamp(rne(fl32(x*r)), -127, 127);
  * an all-zero block gives q = 0 and scale 0.  For K, x = fl32(float(K) - m),
  * m = fl32(double(sum_t int64(K*2^24)) * 2^-24 / Lk), exact and
@@ -91,15 +97,14 @@ SAGE_API sage_status sage_quant_qk(const void *q, const void *k,
                           int8_t *q_i8, int8_t *k_i8,
                           float *q_scale, float *k_scale, float *k_mean,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
-                          float sm_scale, void *workspace, size_t workspace_bytes,
-                          void *stream);
+                          float sm_scale, void *stream);
 
 /*
  * sage_quant_qk_qblock -- sage_quant_qk with a finer Q granularity.
  *
  * The list of techniques in "Berkeley AI 转发研究注意力计算 8 位、4 位量化可对齐
- * FP32 精度基线" (the key-points list) and the SageAttention2 description in
- * the SageAttention article name quantization blocks smaller than the
+ * FP32 精度基线" (the key-points list) and the SageAttention2 entry of the
+ * INT4 search results page name quantization blocks smaller than the
  * attention tile; here Q blocks of q_block_rows rows, one of 128 (the tile,
  * identical to sage_quant_qk), 64, 32 or 1 (one scale per query token).
  * Every block lies inside one 128-row attention tile, so the tiles and the
@@ -114,8 +119,7 @@ SAGE_API sage_status sage_quant_qk_qblock(const void *q, const void *k,
                           int8_t *q_i8, int8_t *k_i8,
                           float *q_scale, float *k_scale, float *k_mean,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
-                          float sm_scale, int q_block_rows,
-                          void *workspace, size_t workspace_bytes, void *stream);
+                          float sm_scale, int q_block_rows, void *stream);
 
 /*
  * sage_quant_k -- steps 1-2 alone: K smoothing (mean over each (batch, kv
@@ -128,15 +132,10 @@ SAGE_API sage_status sage_quant_qk_qblock(const void *q, const void *k,
  *   k_i8     int8 [B, Hkv, Lk, d]          (out)
  *   k_scale  fp32 [B, Hkv, ceil(Lk/64)]    (out)
  *   k_mean   fp32 [B, Hkv, d]              (out)
- *   workspace, workspace_bytes: as sage_quant_qk (sage_quant_workspace_size).
- * Errors: as sage_quant_qk.
+ * No scratch memory.  Errors (and the Lk limit): as sage_quant_qk.
  */
 SAGE_API sage_status sage_quant_k(const void *k, int8_t *k_i8, float *k_scale, float *k_mean,
-                          int B, int Hkv, int Lk, int d,
-                          void *workspace, size_t workspace_bytes, void *stream);
-
-/* Bytes of scratch sage_quant_qk needs (currently 0). */
-SAGE_API size_t sage_quant_workspace_size(int B, int Hkv, int Lk, int d);
+                          int B, int Hkv, int Lk, int d, void *stream);
 
 /*
  * sage_attn_fwd_prequant -- steps 3-5 on already-quantized Q/K: one fused
@@ -171,7 +170,7 @@ SAGE_API sage_status sage_attn_fwd_prequant_qblock(const int8_t *q_i8, const int
  * sage_attn_fwd -- the whole forward pass (steps 1-5) on fp16 Q, K, V.
  *   q fp16 [B, H, Lq, d], k/v fp16 [B, Hkv, Lk, d], out fp16 [B, H, Lq, d].
  * Scratch (int8 Q/K, scales, mean, partial sums;
- * sage_attn_workspace_size() bytes) is allocated with cudaMallocAsync on
+ * sage_workspace_size() bytes) is allocated with cudaMallocAsync on
  * `stream` and released with cudaFreeAsync on the same stream.
  */
 SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, void *out,
@@ -182,7 +181,7 @@ SAGE_API sage_status sage_attn_fwd(const void *q, const void *k, const void *v, 
  * sage_attn_fwd_qblock -- sage_attn_fwd with Q quantized in blocks of
  * q_block_rows rows (128, 64, 32 or 1; see sage_quant_qk_qblock).  Its
  * scratch, allocated and released on `stream` like sage_attn_fwd's, is at
- * most sage_attn_workspace_size() + 4*B*H*Lq + 256 bytes (the Q scales grow
+ * most sage_workspace_size() + 4*B*H*Lq + 256 bytes (the Q scales grow
  * to ceil(Lq/q_block_rows) per head).
  */
 SAGE_API sage_status sage_attn_fwd_qblock(const void *q, const void *k, const void *v, void *out,
@@ -250,8 +249,7 @@ SAGE_API sage_status sage_quant_qk_varlen(const void *q, const void *k,
                           float *q_scale, float *k_scale, float *k_mean,
                           const int *seqlens_q, const int *seqlens_k,
                           int B, int H, int Hkv, int Lq, int Lk, int d,
-                          float sm_scale, int q_block_rows,
-                          void *workspace, size_t workspace_bytes, void *stream);
+                          float sm_scale, int q_block_rows, void *stream);
 SAGE_API sage_status sage_attn_fwd_prequant_varlen(const int8_t *q_i8, const int8_t *k_i8,
                                    const float *q_scale, const float *k_scale,
                                    const void *v, void *out,
@@ -389,6 +387,17 @@ SAGE_API sage_status sage_attn_fwd_host(const void *q_host, const void *k_host, 
                                int causal, float sm_scale, void *stream);
 
 /*
+ * sage_attn_fwd_host_qblock -- sage_attn_fwd_host with Q quantized in blocks
+ * of q_block_rows rows (128, 64, 32 or 1; see sage_quant_qk_qblock); the
+ * output is that of sage_attn_fwd_qblock, bit for bit.  Any other
+ * q_block_rows returns SAGE_ERR_INVALID_ARG.
+ */
+SAGE_API sage_status sage_attn_fwd_host_qblock(const void *q_host, const void *k_host,
+                               const void *v_host, void *out_host,
+                               int B, int H, int Hkv, int Lq, int Lk, int d,
+                               int causal, float sm_scale, int q_block_rows, void *stream);
+
+/*
  * sage_attn_fwd_noalloc -- sage_attn_fwd for callers that must not allocate
  * device memory at call time (a serving process that reserved its whole
  * memory budget at start-up and treats any later allocation as an error, or a
@@ -397,19 +406,27 @@ SAGE_API sage_status sage_attn_fwd_host(const void *q_host, const void *k_host, 
  *   Arguments, layouts and results are those of sage_attn_fwd.  The scratch
  *   lives in one fixed 64 MiB device array inside the library, reserved on
  *   every GPU that loads that part of the library and held until exit.
- *   Problems needing more scratch than that (sage_attn_workspace_size() >
+ *   Problems needing more scratch than that (sage_workspace_size() >
  *   64 MiB) return SAGE_ERR_INVALID_ARG without launching anything.
  *   All calls share the array: calls whose kernels overlap on the GPU race
  *   and give wrong results, so order them on one stream.  The first call on
- *   each device looks the array up; make it before any stream capture begins.
- *   Nothing in the array needs clearing between calls.
+ *   each device (and the first after its context was destroyed and created
+ *   again, e.g. by cudaDeviceReset) looks the array up; make it before any
+ *   stream capture begins.  Nothing in the array needs clearing between
+ *   calls.  Shapes, pointers, scalars and the Lk limit are checked as for
+ *   sage_attn_fwd, and sage_last_launch_count() reports the kernels a
+ *   successful call launched.
  */
 SAGE_API sage_status sage_attn_fwd_noalloc(const void *q, const void *k, const void *v,
                                            void *out, int B, int H, int Hkv, int Lq, int Lk,
                                            int d, int causal, float sm_scale, void *stream);
 
-/* Bytes of scratch sage_attn_fwd allocates for one call. */
-SAGE_API size_t sage_attn_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
+/*
+ * sage_workspace_size -- bytes of device scratch sage_attn_fwd allocates for
+ * one call on this shape (int8 Q and K, their block scales and the K mean,
+ * each piece 256-byte aligned); 0 for a shape the calls reject.
+ */
+SAGE_API size_t sage_workspace_size(int B, int H, int Hkv, int Lq, int Lk, int d);
 
 /*
  * sage_check_device_status -- synchronizes `stream`, then reports and clears

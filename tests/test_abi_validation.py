@@ -19,12 +19,12 @@ OK_, INVALID, UNSUPPORTED = 0, 1, 2
 
 
 def quant_k(k=A, ki=A, ks=A, km=A, B=1, Hkv=2, Lk=128, d=64):
-    return sage.load_library().sage_quant_k(k, ki, ks, km, B, Hkv, Lk, d, N, 0, S)
+    return sage.load_library().sage_quant_k(k, ki, ks, km, B, Hkv, Lk, d, S)
 
 
 def quant_qk_varlen(q=A, qs=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, sm=0.125, qbr=128):
     return sage.load_library().sage_quant_qk_varlen(q, A, A, A, qs, A, A, A, A, B, H, Hkv, Lq,
-                                                    Lk, d, sm, qbr, N, 0, S)
+                                                    Lk, d, sm, qbr, S)
 
 
 def fwd_varlen(out=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, causal=0, sm=0.125, qbr=128,
@@ -36,6 +36,35 @@ def fwd_varlen(out=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, causal=0, sm=0.125,
 def prequant_varlen(qbr=128, flags=0, causal=0):
     return sage.load_library().sage_attn_fwd_prequant_varlen(A, A, A, A, A, A, A, A, 1, 2, 2,
                                                              128, 128, 64, causal, qbr, flags, S)
+
+
+def quant_qk(Lk=128, d=64):
+    return sage.load_library().sage_quant_qk(A, A, A, A, A, A, A, 1, 2, 2, 128, Lk, d, 0.125, S)
+
+
+def quant_qk_qblock(Lk=128, qbr=1):
+    return sage.load_library().sage_quant_qk_qblock(A, A, A, A, A, A, A, 1, 2, 2, 128, Lk, 64,
+                                                    0.125, qbr, S)
+
+
+def fwd(Lk=128, H=2, Lq=128):
+    return sage.load_library().sage_attn_fwd(A, A, A, A, 1, H, 2, Lq, Lk, 64, 0, 0.125, S)
+
+
+def fwd_host(Lk=128):
+    return sage.load_library().sage_attn_fwd_host(A, A, A, A, 1, 2, 2, 128, Lk, 64, 0, 0.125, S)
+
+
+def decode(Lk=1024):
+    return sage.load_library().sage_attn_decode(A, A, A, A, 1, 8, 2, 1, Lk, 128, 1, 0.125, 1, S)
+
+
+def noalloc(q=A, out=A, B=1, H=2, Hkv=2, Lq=128, Lk=128, d=64, causal=0, sm=0.125):
+    return sage.load_library().sage_attn_fwd_noalloc(q, A, A, out, B, H, Hkv, Lq, Lk, d, causal,
+                                                     sm, S)
+
+
+LONG_K = (1 << 20) + 1   # one key past the quantizing calls' limit
 
 
 def quant_v_fp8(v8t=A, vs=A, d=64, Lk=128):
@@ -89,6 +118,29 @@ CASES = [
     ("paged: 16 heads x 9 queries > one tile", lambda: decode_paged(H=16, Hkv=1, Lq=9),
      UNSUPPORTED),
     ("paged: H % Hkv != 0", lambda: decode_paged(H=6, Hkv=4), INVALID),
+    # the Lk limit of the calls that smooth and quantize K
+    ("quant_qk: Lk over the limit", lambda: quant_qk(Lk=LONG_K), UNSUPPORTED),
+    ("quant_qk_qblock: Lk over the limit", lambda: quant_qk_qblock(Lk=LONG_K), UNSUPPORTED),
+    ("quant_qk_varlen: Lk over the limit", lambda: quant_qk_varlen(Lk=LONG_K), UNSUPPORTED),
+    ("quant_k: Lk over the limit", lambda: quant_k(Lk=LONG_K), UNSUPPORTED),
+    ("fwd: Lk over the limit", lambda: fwd(Lk=LONG_K), UNSUPPORTED),
+    ("fwd_varlen: Lk over the limit", lambda: fwd_varlen(Lk=LONG_K), UNSUPPORTED),
+    ("fwd_host: Lk over the limit", lambda: fwd_host(Lk=LONG_K), UNSUPPORTED),
+    ("decode: Lk over the limit", lambda: decode(Lk=LONG_K), UNSUPPORTED),
+    ("noalloc: Lk over the limit", lambda: noalloc(Lk=LONG_K), UNSUPPORTED),
+    # shapes whose element counts do not fit the kernels' index types
+    ("fwd: over 2^40 query elements", lambda: fwd(H=1024, Lq=(1 << 31) - 1), INVALID),
+    ("noalloc: huge B*H", lambda: noalloc(B=1 << 20, H=1 << 10, Hkv=1 << 10), INVALID),
+    # the no-allocation entry point checks what sage_attn_fwd checks
+    ("noalloc: H % Hkv != 0", lambda: noalloc(H=3), INVALID),
+    ("noalloc: d = 96", lambda: noalloc(d=96), UNSUPPORTED),
+    ("noalloc: null q", lambda: noalloc(q=N), INVALID),
+    ("noalloc: misaligned out", lambda: noalloc(out=M), INVALID),
+    ("noalloc: causal 2", lambda: noalloc(causal=2), INVALID),
+    ("noalloc: sm_scale nan", lambda: noalloc(sm=math.nan), INVALID),
+    ("noalloc: sm_scale -1", lambda: noalloc(sm=-1.0), INVALID),
+    ("noalloc: scratch over 64 MiB", lambda: noalloc(H=64, Hkv=64, Lq=4096, Lk=4096, d=128),
+     INVALID),
 ]
 
 

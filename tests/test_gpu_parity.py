@@ -7,7 +7,10 @@ where |O| >= 16, because the output format itself cannot resolve 1e-2 there)
 and cosine >= 0.9999, and full-precision fp64 attention to cosine >= 0.999.
 Small cases compare every element; the full-size workloads compare a seeded
 sample of query rows that includes the first and last rows of every head and
-both sides of each 128-row tile boundary of one head.
+both sides of each 128-row tile boundary of one head.  Each workload runs at
+its own Q granularity (128-row blocks, or one row per block for the
+heavy-tailed long-context workload, whose 128-row blocks miss the fp64 gate;
+that 128-row result is printed, not asserted against the gate).
 """
 import functools
 import math
@@ -56,24 +59,20 @@ def assert_close(gpu_f16, sim, fp64=None, what=""):
     assert c >= COS_SIM, f"{what}: cos vs simulation {c}"
     if fp64 is not None:
         c64 = cos(g, fp64)
-        # The fp64 gate measures the method, not the kernel.  Where the
-        # method's own simulation falls short of it (heavy-tailed inputs), the
-        # kernel must lose nothing relative to that simulation.
-        method = cos(sim, fp64)
-        floor = COS_FP64 if method >= COS_FP64 else method - 1e-4
-        print(f"{what}: cos vs sim {c:.6f}, vs fp64 {c64:.6f} (method {method:.6f})")
-        assert c64 >= floor, f"{what}: cos vs fp64 {c64} (method's own {method})"
+        print(f"{what}: cos vs sim {c:.6f}, vs fp64 {c64:.6f} (method {cos(sim, fp64):.6f})")
+        assert c64 >= COS_FP64, f"{what}: cos vs fp64 {c64}"
+    return c
 
 
-def gpu_quant(q, k, sm):
-    outs = sage.quant_qk(to_dev(q), to_dev(k), sm)
+def gpu_quant(q, k, sm, qbr=128):
+    outs = sage.quant_qk(to_dev(q), to_dev(k), sm, q_block_rows=qbr)
     sage.sage_check_device_status()
     return [t.cpu().numpy() for t in outs]
 
 
-def gpu_attention(q, k, v, causal, sm):
+def gpu_attention(q, k, v, causal, sm, qbr=128):
     torch = torch_mod()
-    out = sage.attention(to_dev(q), to_dev(k), to_dev(v), causal, sm)
+    out = sage.attention(to_dev(q), to_dev(k), to_dev(v), causal, sm, q_block_rows=qbr)
     sage.sage_check_device_status()
     return out.cpu().numpy()
 
@@ -188,6 +187,21 @@ def test_host_buffer_entry_point_matches_device(shape):
     assert torch.equal(hout, dev.cpu())
 
 
+def test_host_buffer_entry_point_with_finer_q_blocks():
+    """sage_attn_fwd_host_qblock equals the device call at the same Q
+    granularity, bit for bit."""
+    torch = torch_mod()
+    q, k, v = inputs.make_custom(2, 8, 4, 300, 400, 128, seed=17)
+    hq, hk, hv = (torch.from_numpy(x).pin_memory() for x in (q, k, v))
+    for qbr in (1, 32):
+        hout = torch.empty(q.shape, dtype=torch.float16).pin_memory()
+        sage.sage_attn_fwd_host_qblock(hq, hk, hv, hout, True, 0.088, qbr)
+        torch.cuda.current_stream().synchronize()
+        dev = sage.attention(to_dev(q), to_dev(k), to_dev(v), True, 0.088, q_block_rows=qbr)
+        sage.sage_check_device_status()
+        assert torch.equal(hout, dev.cpu()), qbr
+
+
 # ------------------------------------------------------------ closed forms
 
 @pytest.mark.parametrize("causal", [False, True])
@@ -250,19 +264,41 @@ def workload_data(idx):
 
 @pytest.mark.parametrize("idx", [1, 2, 3, 4, 5])
 def test_workload(idx):
-    """Full-size workload through sage_attn_fwd: quantization bit-exact over
-    every element, output checked on the seeded row sample (all rows for the
-    tiny workload)."""
+    """Full-size workload through sage_attn_fwd at the workload's Q
+    granularity: quantization bit-exact over every element, output checked
+    on the seeded row sample (all rows for the tiny workload), fp64 gate
+    unrelaxed."""
     w, q, k, v = workload_data(idx)
+    sm = float(np.float32(w.sm_scale))
+    qbr = w.q_block_rows
+    want_q = oracle.quant_qk(q, k, sm, q_block_rows=qbr)
+    assert_quant_bitexact(gpu_quant(q, k, sm, qbr), want_q, w.name)
+    out = gpu_attention(q, k, v, w.causal, sm, qbr).reshape(-1, w.d)
+    rows = None if idx == 1 else inputs.sample_rows(w.B, w.H, w.Lq, 512, seed=idx)
+    sim = oracle.attn_quant_sim(*want_q[:4], v, w.causal, rows=rows,
+                                q_block_rows=qbr).reshape(-1, w.d)
+    ref = oracle.attn_fp64(q, k, v, w.causal, sm, rows=rows).reshape(-1, w.d)
+    got = out if rows is None else out[rows]
+    assert_close(got, sim, ref, f"{w.name} (Q blocks of {qbr})")
+
+
+def test_longctx_tile_granularity_reported():
+    """The long-context workload at 128-row Q blocks (the attention tile):
+    the kernel must match the oracle's simulation of that granularity; its
+    accuracy against fp64 attention is printed as a reported number (the
+    method itself falls short of 0.999 there, which is why the workload runs
+    with per-token Q blocks)."""
+    w, q, k, v = workload_data(5)
     sm = float(np.float32(w.sm_scale))
     want_q = oracle.quant_qk(q, k, sm)
     assert_quant_bitexact(gpu_quant(q, k, sm), want_q, w.name)
     out = gpu_attention(q, k, v, w.causal, sm).reshape(-1, w.d)
-    rows = None if idx == 1 else inputs.sample_rows(w.B, w.H, w.Lq, 512, seed=idx)
+    rows = inputs.sample_rows(w.B, w.H, w.Lq, 512, seed=5)
     sim = oracle.attn_quant_sim(*want_q[:4], v, w.causal, rows=rows).reshape(-1, w.d)
     ref = oracle.attn_fp64(q, k, v, w.causal, sm, rows=rows).reshape(-1, w.d)
-    got = out if rows is None else out[rows]
-    assert_close(got, sim, ref, w.name)
+    assert_close(out[rows], sim, None, f"{w.name} (Q blocks of 128)")
+    print(f"{w.name} with 128-row Q blocks: cos vs fp64 {cos(out[rows], ref):.6f} "
+          f"(method {cos(sim, ref):.6f}; reported, not gated)")
 
 
 def test_degenerate_blocks_zero_q_and_constant_k():

@@ -7,9 +7,13 @@ the test makes two calls in a row with different problems (the second must
 not see anything the first left behind) and checks each against the regular
 sage_attn_fwd, within the parity tolerance the other GPU tests use.  It also
 checks that a problem too large for the array is refused without touching the
-output.  This file is collected last and must pass both alone in a fresh
-process and after the other tests.
+output, and that a warm call really allocates nothing: the high-water mark of
+the device's default memory pool (where cudaMallocAsync takes memory) does
+not move across two no-allocation calls, while the same instrument does see
+the allocating entry point's scratch.  This file is collected last and must
+pass both alone in a fresh process and after the other tests.
 """
+import ctypes
 import math
 
 import numpy as np
@@ -53,7 +57,7 @@ def test_noalloc_matches_allocating_entry_point_twice_in_a_row():
         ((2, 8, 2, 700, 900, 64), False, 12),        # different shape, GQA, ragged tails
     ]
     for (B, H, Hkv, Lq, Lk, d), causal, seed in cases:
-        assert sage.sage_attn_workspace_size(B, H, Hkv, Lq, Lk, d) <= sage.NOALLOC_SCRATCH_BYTES
+        assert sage.sage_workspace_size(B, H, Hkv, Lq, Lk, d) <= sage.NOALLOC_SCRATCH_BYTES
         q, k, v = _problem(B, H, Hkv, Lq, Lk, d, seed)
         sm = 1.0 / math.sqrt(d)
         out_fixed = torch.full_like(q, float("nan"))
@@ -68,7 +72,7 @@ def test_noalloc_matches_allocating_entry_point_twice_in_a_row():
 def test_noalloc_refuses_problems_larger_than_its_array():
     torch = _torch()
     B, H, Hkv, L, d = 1, 64, 64, 4096, 128      # ~68 MB of scratch
-    assert sage.sage_attn_workspace_size(B, H, Hkv, L, L, d) > sage.NOALLOC_SCRATCH_BYTES
+    assert sage.sage_workspace_size(B, H, Hkv, L, L, d) > sage.NOALLOC_SCRATCH_BYTES
     q = torch.zeros((B, H, L, d), dtype=torch.float16, device="cuda")
     out = torch.full_like(q, 7.0)
     with pytest.raises(sage.SageError) as e:
@@ -76,3 +80,63 @@ def test_noalloc_refuses_problems_larger_than_its_array():
     assert e.value.status == 1
     torch.cuda.synchronize()
     assert bool((out == 7.0).all())
+
+
+# CUmemPool_attribute values (cuda.h): memory of the pool in use now, and its
+# high-water mark since the last reset (setting it to 0 resets it to "now").
+CU_MEMPOOL_ATTR_USED_MEM_CURRENT = 7
+CU_MEMPOOL_ATTR_USED_MEM_HIGH = 8
+
+
+class _DefaultPool:
+    """The current device's default memory pool, through the driver API."""
+
+    def __init__(self):
+        self.cu = ctypes.CDLL("libcuda.so.1")
+        dev = ctypes.c_int()
+        assert self.cu.cuCtxGetDevice(ctypes.byref(dev)) == 0
+        self.pool = ctypes.c_void_p()
+        assert self.cu.cuDeviceGetDefaultMemPool(ctypes.byref(self.pool), dev) == 0
+
+    def _get(self, attr):
+        v = ctypes.c_uint64()
+        assert self.cu.cuMemPoolGetAttribute(self.pool, attr, ctypes.byref(v)) == 0
+        return v.value
+
+    def used(self):
+        return self._get(CU_MEMPOOL_ATTR_USED_MEM_CURRENT)
+
+    def high(self):
+        return self._get(CU_MEMPOOL_ATTR_USED_MEM_HIGH)
+
+    def reset_high(self):
+        z = ctypes.c_uint64(0)
+        assert self.cu.cuMemPoolSetAttribute(self.pool, CU_MEMPOOL_ATTR_USED_MEM_HIGH,
+                                             ctypes.byref(z)) == 0
+
+
+def test_noalloc_warm_calls_take_no_device_memory():
+    torch = _torch()
+    B, H, Hkv, L, d = 1, 8, 8, 2048, 128
+    q, k, v = _problem(B, H, Hkv, L, L, d, seed=13)
+    out = torch.empty_like(q)
+    sage.sage_attn_fwd_noalloc(q, k, v, out, True, 0.088)      # warm: first-call set-up
+    sage.sage_attn_fwd(q, k, v, out, True, 0.088)
+    torch.cuda.synchronize()
+    pool = _DefaultPool()
+    # control: the instrument sees the allocating entry point's scratch
+    pool.reset_high()
+    base = pool.high()
+    sage.sage_attn_fwd(q, k, v, out, True, 0.088)
+    torch.cuda.synchronize()
+    assert pool.high() >= base + sage.sage_workspace_size(B, H, Hkv, L, L, d)
+    # the no-allocation entry point: two calls, no pool memory at all
+    pool.reset_high()
+    base = pool.high()
+    assert base == pool.used()
+    for _ in range(2):
+        sage.sage_attn_fwd_noalloc(q, k, v, out, True, 0.088)
+        assert sage.sage_last_launch_count() == 2
+    torch.cuda.synchronize()
+    assert pool.high() == base
+    sage.sage_check_device_status()
