@@ -59,16 +59,24 @@ __device__ __forceinline__ void block_absmax_n(float (&v)[NB], float* red) {
   __syncthreads();  // red[] may be reused by the next group of blocks
 }
 
-// rne(fl32(x * r)) clamped to [-127, 127], as an int.  The rounding adds
-// 1.5 * 2^23 in fp32 (the FADD itself rounds to the nearest integer, ties to
-// even, exactly as cvt.rni would for |x * r| < 2^22) and reads the integer
-// back from the low mantissa bits; this keeps the conversion off the
-// transcendental/conversion unit.
-__device__ __forceinline__ int quant_one(float x, float r) {
-  const float y = __fmul_rn(x, r);
-  const float big = __fadd_rn(y, 12582912.f);
-  const int t = __float_as_int(big) - 0x4B400000;
-  return max(-127, min(127, t));
+// The int8 codes rne(fl32(x * r)) of 8 values, packed low byte first.  The
+// rounding adds 1.5 * 2^23 in fp32: the FADD itself rounds to the nearest
+// integer q (ties to even, as cvt.rni would for |x * r| < 2^22), and the sum's
+// bit pattern is 0x4B400000 + q, whose low byte is q's two's-complement code.
+// No clamp is needed: every caller has |x| <= a and r = fl32(127 / a), so
+// |fl32(x * r)| <= 127 (1 + 2^-24)^2 < 127.5 and |q| <= 127.
+// Scalar IEEE operations throughout: the paired fp32 instructions of sm_100
+// were measured to round some exact ties (x = a / 2, fl32(x * r) = 63.5)
+// differently from round-half-to-even.
+__device__ __forceinline__ uint2 quant8(const float (&x)[8], float r) {
+  uint32_t w[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) w[e] = __float_as_uint(__fadd_rn(__fmul_rn(x[e], r), 12582912.f));
+  const uint32_t lo = __byte_perm(__byte_perm(w[0], w[1], 0x0040), __byte_perm(w[2], w[3], 0x0040),
+                                  0x5410);
+  const uint32_t hi = __byte_perm(__byte_perm(w[4], w[5], 0x0040), __byte_perm(w[6], w[7], 0x0040),
+                                  0x5410);
+  return make_uint2(lo, hi);
 }
 
 __device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
@@ -81,7 +89,7 @@ __device__ __forceinline__ void unpack8(const uint4& u, float (&x)[8]) {
   }
 }
 
-// Smoothed (for K) fp32 values of one 16-byte vector.
+// fp32 values of one 16-byte vector of fp16, smoothed for K: fl32(float(K) - m).
 template <bool SMOOTH>
 __device__ __forceinline__ void values8(const uint4& raw, const float (&m)[8], float (&x)[8]) {
   unpack8(raw, x);
@@ -89,6 +97,22 @@ __device__ __forceinline__ void values8(const uint4& raw, const float (&m)[8], f
 #pragma unroll
     for (int e = 0; e < 8; ++e) x[e] = __fsub_rn(x[e], m[e]);
   }
+}
+
+// max |h| over the 8 fp16 values of a 16-byte vector, folded into a running
+// (max, min) pair of fp16x2 accumulators (exact: fp16 max/min).
+__device__ __forceinline__ void absmax8_h(const uint4& u, __half2& mx, __half2& mn) {
+  const __half2* h = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    mx = __hmax2(mx, h[e]);
+    mn = __hmin2(mn, h[e]);
+  }
+}
+
+__device__ __forceinline__ float absmax_of(const __half2& mx, const __half2& mn) {
+  const float2 a = __half22float2(mx), b = __half22float2(mn);
+  return fmaxf(fmaxf(a.x, a.y), fmaxf(-b.x, -b.y));
 }
 
 // Quantizes one 128-row Q tile whose quantization blocks are QBR rows
@@ -114,17 +138,18 @@ __device__ __forceinline__ void quant_q_tile(const __half* __restrict__ src, int
   }
   const float no_mean[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   float amax[NG];
+  {
+    __half2 mx[NG], mn[NG];
 #pragma unroll
-  for (int g = 0; g < NG; ++g) amax[g] = 0.f;
+    for (int g = 0; g < NG; ++g) mx[g] = mn[g] = __float2half2_rn(0.f);
 #pragma unroll
-  for (int v = 0; v < VPT; ++v) {
-    if (tid + v * kQuantThreads < nvec) {
-      float x[8];
-      values8<false>(raw[v], no_mean, x);
+    for (int v = 0; v < VPT; ++v) {
       const int g = QBR == 1 ? v : v / (QBR / RPP);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) amax[g] = fmaxf(amax[g], fabsf(x[e]));
+      // rows past the tile were loaded as zeros: they do not change the max
+      absmax8_h(raw[v], mx[g], mn[g]);
     }
+#pragma unroll
+    for (int g = 0; g < NG; ++g) amax[g] = absmax_of(mx[g], mn[g]);
   }
   if (QBR == 1) {
     // the TPR lanes of one row are adjacent within a warp
@@ -145,12 +170,7 @@ __device__ __forceinline__ void quant_q_tile(const __half* __restrict__ src, int
     if (idx < nvec) {
       float x[8];
       values8<false>(raw[v], no_mean, x);
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
-      __stcs(reinterpret_cast<uint2*>(dst) + idx, make_uint2(lo, hi));
+      __stcs(reinterpret_cast<uint2*>(dst) + idx, quant8(x, r));
     }
     // one thread per block writes its scale
     const int row = idx / TPR;
@@ -208,12 +228,7 @@ __device__ __forceinline__ void quant_k_blocks(const __half* __restrict__ kh, in
       if (idx < nvec[b]) {
         float x[8];
         values8<true>(raw[b][v], m, x);
-        uint32_t lo = 0, hi = 0;
-#pragma unroll
-        for (int e = 0; e < 4; ++e) lo |= (uint32_t)(quant_one(x[e], r) & 0xff) << (8 * e);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) hi |= (uint32_t)(quant_one(x[4 + e], r) & 0xff) << (8 * e);
-        __stcs(dst + idx, make_uint2(lo, hi));
+        __stcs(dst + idx, quant8(x, r));
       }
     }
     if (tid == 0 && nvec[b] > 0) ks[kb + b] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
@@ -223,7 +238,7 @@ __device__ __forceinline__ void quant_k_blocks(const __half* __restrict__ kh, in
 // ------------------------------------------------------------- kernel
 
 template <int D, int QBR>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, 4)
 quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
                 int8_t* __restrict__ q_i8, int8_t* __restrict__ k_i8,
                 float* __restrict__ q_scale, float* __restrict__ k_scale,
@@ -276,10 +291,14 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
 #pragma unroll 8
     for (int t = t0 + rr; t < t1; t += RPP) {
-      float x[8];
-      unpack8(__ldg(base + (size_t)t * TPR), x);
+      const uint4 u = __ldg(base + (size_t)t * TPR);
+      const unsigned short* h = reinterpret_cast<const unsigned short*>(&u);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += (double)x[e];
+      for (int e = 0; e < 8; ++e) {
+        double x;  // fp16 -> fp64 is exact
+        asm("cvt.f64.f16 %0, %1;" : "=d"(x) : "h"(h[e]));
+        acc[e] += x;
+      }
     }
     // fp16 values are multiples of 2^-24 below 2^16: each double sum of at
     // most 2^13 of them is exact, and so is its conversion to int64
