@@ -11,8 +11,12 @@
 //     thread, then int64 counts of 2^-24); the cluster then adds the
 //     kCluster partial sums through distributed shared memory in a fixed
 //     order, so every CTA holds the same exact mean (rank 0 stores it).
-//     Pass 2 re-reads its rows (from L2), subtracts the mean and quantizes
-//     its 64-row blocks, two at a time.
+//     At d = 64 pass 1 also keeps each block's per-channel fp16 minimum and
+//     maximum: rounding is monotonic, so with the mean known they give the
+//     block's abs-max of fl32(K - mean) exactly, and pass 2 re-reads the rows
+//     as one barrier-free stream (subtract, scale, round, store).  Otherwise
+//     (d = 128, or more blocks than shared memory holds extremes for) pass 2
+//     quantizes two blocks at a time, each reduced across the CTA.
 //   * Q clusters: every CTA quantizes one 128-row Q block (Q does not depend
 //     on the mean, so this overlaps the K work).
 //
@@ -252,6 +256,9 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   __shared__ long long part[D];   // this CTA's exact column sums (units of 2^-24)
   __shared__ long long rsum[RPP * D > 0 ? RPP * D : 1];
   __shared__ float mean[D];
+  // per-block channel max and min of K, and 127 / abs-max (d = 64 path)
+  __shared__ __half2 kext[D == 64 ? 4096 : 1];
+  __shared__ float kr[D == 64 ? 4096 / D : 1];
   const int tid = threadIdx.x;
 
   if ((int)blockIdx.x >= n_k_ctas) {
@@ -282,16 +289,30 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   const int t0 = kb0 * SAGE_K_BLOCK_ROWS, t1 = min(Lkb, kb1 * SAGE_K_BLOCK_ROWS);
   const __half* kh = k + (size_t)bhk * Lk * D;
 
-  // pass 1: exact column sums of rows [t0, t1)
+  // Per-block channel extremes, kept when this CTA's blocks fit in kFastBlocks:
+  // fl32 rounding is monotonic, so over a block the largest |fl32(k - m_c)| of
+  // channel c is taken at that channel's smallest or largest k.  Once the mean
+  // is known the block abs-max (and so the block scale) follows exactly,
+  // without a second pass over the rows.
+  // Used at d = 64, where it measured 8 % faster; at d = 128 the extra
+  // registers it needs cost the Q tiles (one kernel, one register budget)
+  // more than the shorter second pass gains.
+  constexpr bool kExtremes = D == 64;
+  constexpr int kFastBlocks = kExtremes ? 4096 / D : 0;
+  const int nb = kb1 - kb0;
+  const bool fast = kExtremes && nb <= kFastBlocks;
+  constexpr int R = 32 / TPR;  // rows per warp-wide load (each lane: one 16-byte vector)
+  const int warp = tid >> 5, lane = tid & 31;
+  const int sub = lane / TPR, cg8 = lane % TPR;
+
+  // pass 1: exact column sums of rows [t0, t1).  Lane (sub, cg8) of warp w
+  // is row class rr = w * R + sub = tid / TPR for the channels of cg8.
   {
-    const int cg8 = tid % TPR, rr = tid / TPR;
     const uint4* base = reinterpret_cast<const uint4*>(kh) + cg8;
     double acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0;
-#pragma unroll 8
-    for (int t = t0 + rr; t < t1; t += RPP) {
-      const uint4 u = __ldg(base + (size_t)t * TPR);
+    auto add8 = [&](const uint4& u) {
       const unsigned short* h = reinterpret_cast<const unsigned short*>(&u);
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -299,9 +320,57 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
         asm("cvt.f64.f16 %0, %1;" : "=d"(x) : "h"(h[e]));
         acc[e] += x;
       }
+    };
+    if constexpr (!kExtremes) {
+      // row class rr takes every RPP-th row
+#pragma unroll 8
+      for (int t = t0 + tid / TPR; t < t1; t += RPP) add8(__ldg(base + (size_t)t * TPR));
+    } else {
+      // warp w takes whole blocks w, w + 8, ... and their channel extremes
+      for (int bl = warp; bl < nb; bl += kQuantThreads / 32) {
+        const int r0 = t0 + bl * SAGE_K_BLOCK_ROWS;
+        const int r1 = min(t1, r0 + SAGE_K_BLOCK_ROWS);
+        __half2 mx[4], mn[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          mx[e] = __float2half2_rn(-INFINITY);
+          mn[e] = __float2half2_rn(INFINITY);
+        }
+#pragma unroll 8
+        for (int t = r0 + sub; t < r1; t += R) {
+          const uint4 u = __ldg(base + (size_t)t * TPR);
+          add8(u);
+          const __half2* h2 = reinterpret_cast<const __half2*>(&u);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            mx[e] = __hmax2(mx[e], h2[e]);
+            mn[e] = __hmin2(mn[e], h2[e]);
+          }
+        }
+        if (fast) {
+          // the R lanes holding the same channels are TPR apart
+#pragma unroll
+          for (int o = TPR; o < 32; o <<= 1)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              mx[e] = __hmax2(mx[e], __shfl_xor_sync(0xffffffffu, mx[e], o));
+              mn[e] = __hmin2(mn[e], __shfl_xor_sync(0xffffffffu, mn[e], o));
+            }
+          if (sub == 0) {
+            // block bl: per 8-channel group, 4 fp16x2 maxima then 4 minima
+            __half2* dst = kext + (size_t)bl * D + cg8 * 8;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              dst[e] = mx[e];
+              dst[4 + e] = mn[e];
+            }
+          }
+        }
+      }
     }
     // fp16 values are multiples of 2^-24 below 2^16: each double sum of at
     // most 2^13 of them is exact, and so is its conversion to int64
+    const int rr = warp * R + sub;  // one of RPP row classes
 #pragma unroll
     for (int e = 0; e < 8; ++e) rsum[rr * D + cg8 * 8 + e] = (long long)(acc[e] * 16777216.0);
     __syncthreads();
@@ -321,13 +390,71 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   }
   cluster.sync();  // no CTA leaves (or reuses part[]) while others read it
 
-  // pass 2: smooth and quantize this CTA's K blocks
   float m8[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) m8[e] = mean[(tid % TPR) * 8 + e];
-  for (int kb = kb0; kb < kb1; kb += 2)
-    quant_k_blocks<D, 2>(k + (size_t)bhk * Lk * D, k_i8 + (size_t)bhk * Lk * D,
-                         k_scale + (size_t)bhk * nkb, kb, kb1, Lkb, m8, red);
+  if (!fast) {
+    // pass 2 (d = 128, or more blocks than the extremes cover): re-read,
+    // smooth and quantize two blocks at a time
+    for (int kb = kb0; kb < kb1; kb += 2)
+      quant_k_blocks<D, 2>(k + (size_t)bhk * Lk * D, k_i8 + (size_t)bhk * Lk * D,
+                           k_scale + (size_t)bhk * nkb, kb, kb1, Lkb, m8, red);
+    return;
+  }
+
+  // block scales from the extremes: 8 lanes per block, D/8 channels each; the
+  // loop bound is warp-uniform so every lane reaches the shuffles
+  {
+    constexpr int CPL = D / 8;
+    for (int base = warp * 4; base < nb; base += kQuantThreads / 8) {
+      const int bl = base + lane / 8;
+      float a = 0.f;
+      if (bl < nb) {
+        const __half* ext = reinterpret_cast<const __half*>(kext + (size_t)bl * D);
+        const int c0 = (lane % 8) * CPL;
+#pragma unroll 8
+        for (int c = c0; c < c0 + CPL; ++c) {
+          // channel c: its 8-channel group's maxima, then its minima
+          const int g = (c >> 3) * 16 + (c & 7);
+          const float hi = __half2float(ext[g]), lo = __half2float(ext[g + 8]);
+          a = fmaxf(a, fabsf(__fsub_rn(hi, mean[c])));
+          a = fmaxf(a, fabsf(__fsub_rn(lo, mean[c])));
+        }
+      }
+#pragma unroll
+      for (int o = 4; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
+      if (bl < nb && lane % 8 == 0) {
+        kr[bl] = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+        k_scale[(size_t)bhk * nkb + kb0 + bl] = a > 0.f ? __fdiv_rn(a, 127.f) : 0.f;
+      }
+    }
+  }
+  __syncthreads();
+
+  // pass 2: one stream over the rows [t0, t1): smooth, quantize, store
+  {
+    const int nvec = (t1 - t0) * TPR;
+    const uint4* src = reinterpret_cast<const uint4*>(kh + (size_t)t0 * D);
+    uint2* dst = reinterpret_cast<uint2*>(k_i8 + ((size_t)bhk * Lk + t0) * D);
+    constexpr int U = 8;
+    for (int i0 = tid; i0 < nvec; i0 += U * kQuantThreads) {
+      uint4 raw[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int idx = i0 + u * kQuantThreads;
+        raw[u] = idx < nvec ? __ldcs(src + idx) : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int idx = i0 + u * kQuantThreads;
+        if (idx < nvec) {
+          float x[8];
+          values8<true>(raw[u], m8, x);
+          __stcs(dst + idx, quant8(x, kr[idx / (SAGE_K_BLOCK_ROWS * TPR)]));
+        }
+      }
+    }
+  }
 }
 
 // ------------------------------------------------------------- launcher
@@ -344,10 +471,11 @@ static cudaError_t launch_quant_d(const QuantArgs& a, cudaStream_t st, int* laun
       cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess)
     cl = 16;
   const int kb_per_cta = (nkb + cl - 1) / cl;
-  // a CTA sums at most kb_per_cta * 64 rows and each thread at most 1/RPP of
-  // them, at most 2^13 exact double sums; the entry points refuse Lk above
+  // a CTA sums kb_per_cta blocks of 64 rows, each warp every 8th block and
+  // each lane 1/R of a block's rows (R = 32 / (D / 8)): at most 2^13 exact
+  // double sums per lane; the entry points refuse Lk above
   // SAGE_MAX_LK (2^20), which keeps this bound for every cluster width and d
-  if ((long long)kb_per_cta * SAGE_K_BLOCK_ROWS / (kQuantThreads / (D / 8)) > 8192)
+  if ((long long)(kb_per_cta + 7) / 8 * (SAGE_K_BLOCK_ROWS / (32 / (D / 8))) > 8192)
     return cudaErrorInvalidValue;
   const long long n_k_ctas = (long long)BHkv * cl;
   const long long n_q_blocks = a.skip_q ? 0 : (long long)BH * nqb;

@@ -20,6 +20,10 @@ SHAPES = [
     (1, 2, 2, 260, 70, 64),
     (1, 1, 1, 1, 1, 128),         # a single key
     (1, 8, 8, 1024, 1024, 128),
+    # more K blocks per CTA than the per-block extremes in shared memory
+    # cover (32 at d = 128, 64 at d = 64): the two-blocks-at-a-time pass
+    (1, 1, 1, 1, 40000, 128),
+    (1, 2, 1, 1, 70001, 64),
 ]
 
 
