@@ -35,8 +35,13 @@
 // (O rescaled whenever it grows) so that P <= 1 keeps the sums in fp16 range.
 // The default accumulates in fp32.
 //
+// At d = 64 (fp16 P V, fp32 sums) P V runs with N = d + 16 against V and a
+// constant tile whose first column is all ones, so the accumulator's column d
+// is each row's sum of the same fp16 P the MMA used, and the softmax warps
+// keep no row sum of their own.
+//
 // Tensor memory (256 columns): [0,64) S/P buffer 0, [64,128) S/P buffer 1,
-// [128,128+d) O accumulator.  Every mbarrier wait is bounded (2 s); on expiry
+// [128,128+d) O accumulator (+16 columns, the row sums, at d = 64).  Every mbarrier wait is bounded (2 s); on expiry
 // the CTA stops issuing work, drains what is in flight, frees its tensor
 // memory and records the failing site in the device status word.
 #include <cuda.h>
@@ -63,7 +68,7 @@ constexpr int BK = 64;   // key rows per tile    (= K quantization block)
 // in E4M3 with fp32 sums.
 enum PvMode : int { kPvF32 = 0, kPvF16Acc = 1, kPvFp8 = 2 };
 
-template <int D, bool FP8V = false>
+template <int D, bool FP8V = false, bool ONES = false>
 struct AttnCfg {
   static constexpr int STAGES = 3;
   static constexpr int Q_BYTES = BQ * D;      // int8
@@ -73,7 +78,10 @@ struct AttnCfg {
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + Q_BYTES;
   static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
-  static constexpr int OFF_BAR = OFF_V + STAGES * V_BYTES;
+  // ONES: a constant [64 keys x 64] fp16 tile whose first column is 1, read
+  // as 16 more B columns of P V, so the tensor core also sums P per row
+  static constexpr int OFF_ONES = OFF_V + STAGES * V_BYTES;
+  static constexpr int OFF_BAR = OFF_ONES + (ONES ? BK * 128 : 0);
   // barrier slots
   static constexpr int B_Q_FULL = 0;
   static constexpr int B_K_FULL = 1;
@@ -129,7 +137,11 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const int* __restrict__ seqlens_k) {
   constexpr bool F16ACC = PV == kPvF16Acc;
   constexpr bool FP8V = PV == kPvFp8;
-  using C = AttnCfg<D, FP8V>;
+  // d = 64, fp16 P V with fp32 sums: the row sums of P come from the tensor
+  // core (16 extra accumulator columns, the first one the sum)
+  constexpr bool ONES = D == 64 && PV == kPvF32;
+  constexpr int OW = ONES ? D + 16 : D;  // accumulator columns of P V
+  using C = AttnCfg<D, FP8V, ONES>;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment of the shared-window address (swizzle atoms)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -175,6 +187,16 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   if (warp == 5) {
     tmem_alloc(tmem_slot, C::TMEM_COLS);
     tmem_relinquish();
+  }
+  if constexpr (ONES) {
+    // key row r holds 128 bytes; its 16-byte chunk c sits at chunk c ^ (r % 8)
+    // (128-byte swizzle), so column 0 of row r is at byte r * 128 + (r % 8) * 16
+    uint4* ones = reinterpret_cast<uint4*>(smem + C::OFF_ONES);
+    for (int i = tid; i < BK * 8; i += blockDim.x) {
+      const int r = i >> 3, cchunk = i & 7;
+      ones[i] = make_uint4(cchunk == (r & 7) ? 0x3C00u : 0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();  // visible to the tensor core
   }
   if (warp == 4 && lane == 0) {
     tma_prefetch_desc(&tm_q);
@@ -229,7 +251,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (lane == 0 && nkt > 0) {
       constexpr uint32_t idesc_qk = make_idesc_i8(BQ, BK);
       constexpr uint32_t idesc_pv =
-          FP8V ? make_idesc_f8(BQ, D) : make_idesc_f16(BQ, D, /*b_mn_major=*/true, F16ACC);
+          FP8V ? make_idesc_f8(BQ, D) : make_idesc_f16(BQ, OW, /*b_mn_major=*/true, F16ACC);
       const uint32_t sQ = smem_u32(smem + C::OFF_Q);
       auto issue_pv = [&](int jj) -> bool {
         const int bb = jj & 1, ss = jj % C::STAGES;
@@ -255,8 +277,10 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           for (int kk = 0; kk < BK / 16; ++kk) {
             // V tile: D/64 chunks of [64 keys x 128 B] (128B swizzle), MN-major
             // B operand; LBO = chunk stride, SBO = 8 key rows; 16 keys per MMA.
-            const uint64_t bdesc =
-                make_smem_desc(sV + kk * 16 * 128, BK * 128, 1024, kSwizzle128B);
+            // with ONES the second 64-column atom is the ones tile
+            const uint32_t lbo = ONES ? (uint32_t)(C::OFF_ONES - C::OFF_V - ss * C::V_BYTES)
+                                      : (uint32_t)(BK * 128);
+            const uint64_t bdesc = make_smem_desc(sV + kk * 16 * 128, lbo, 1024, kSwizzle128B);
             umma_f16_ts(tmem + C::O_COL, p_tmem + kk * 8, bdesc, idesc_pv,
                         (jj > 0 || kk > 0) ? 1u : 0u);
           }
@@ -353,7 +377,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         tc_fence_after_sync();
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
+        for (int cc = 0; cc < (OW + 31) / 32; ++cc) {
           uint32_t o[32];
           tmem_ld32(tmem + lane_base + C::O_COL + cc * 32, o);
 #pragma unroll
@@ -377,7 +401,7 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           p0 = k < vis ? p0 : 0.f;
           p1 = k + 1 < vis ? p1 : 0.f;
         }
-        lsum += p0 + p1;
+        if constexpr (!ONES) lsum += p0 + p1;
         if constexpr (FP8V) {
           // P <= 2^8 (lazy max), so P * 1.75 <= 448 fits E4M3; 4 keys a column
           const uint32_t e = pack_e4m3x2(p0 * 1.75f, p1 * 1.75f);
@@ -400,7 +424,14 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       tc_fence_after_sync();
     }
     if (ok) {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float lsum_all = l_run;
+      if constexpr (ONES) {
+        // the tensor core's row sum of the fp16 P, column D of the accumulator
+        uint32_t o[32];
+        if (nkt > 0) tmem_ld32(tmem + lane_base + C::O_COL + D, o);
+        lsum_all = nkt > 0 ? __uint_as_float(o[0]) : 0.f;
+      }
+      const float inv = lsum_all > 0.f ? 1.f / lsum_all : 0.f;
       __half* orow = out + ((size_t)bh * Lq + qrow) * D;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -476,7 +507,7 @@ static bool make_map_3d(CUtensorMap* map, const void* base, CUtensorMapDataType 
 
 template <int D, bool CAUSAL, int PV>
 static cudaError_t launch_attn_t(const AttnArgs& a, cudaStream_t st, int* launches) {
-  using C = AttnCfg<D, PV == kPvFp8>;
+  using C = AttnCfg<D, PV == kPvFp8, D == 64 && PV == kPvF32>;
   auto kern = sage_attn_fwd_kernel<D, CAUSAL, PV>;
   // per device context; cheap enough to repeat on every launch
   cudaError_t attr_err =
