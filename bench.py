@@ -67,8 +67,8 @@ EX2_PER_CLK_PER_SM = 16  # MUFU ex2 results per clock per SM (measured 15.9)
 
 # DRAM traffic of one attention launch from an ncu capture, valid only for the
 # kernel source it was taken on (attn_source_hash); otherwise reported null.
-NCU_TRAFFIC = {"attn_sha": "0426d895995a5473", "workload": "longctx-causal-B1H16L32768d128-t4",
-               "q_block_rows": 1, "bytes_per_launch": 271057920 + 108540928}
+NCU_TRAFFIC = {"attn_sha": "11cca823bf95dac9", "workload": "longctx-causal-B1H16L32768d128-t4",
+               "q_block_rows": 1, "bytes_per_launch": 270883840 + 106859008}
 # Same for the decoding kernel (decode.cu + PTX wrappers) on the --decode shape.
 DECODE_NCU_TRAFFIC = {"sha": "6a43014109bd395c", "bytes_per_launch": 805530880 + 3755520}
 
