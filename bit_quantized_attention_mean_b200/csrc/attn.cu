@@ -41,9 +41,10 @@
 // keep no row sum of their own.
 //
 // Tensor memory (256 columns): [0,64) S/P buffer 0, [64,128) S/P buffer 1,
-// [128,128+d) O accumulator (+16 columns, the row sums, at d = 64).  Every mbarrier wait is bounded (2 s); on expiry
-// the CTA stops issuing work, drains what is in flight, frees its tensor
-// memory and records the failing site in the device status word.
+// [128,128+d) O accumulator (+16 columns, the row sums, at d = 64).  Every
+// mbarrier wait is bounded (2 s); on expiry the CTA stops issuing work, drains
+// what is in flight, frees its tensor memory and records the failing site in
+// the device status word.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
@@ -376,6 +377,8 @@ sage_attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           break;
         }
         tc_fence_after_sync();
+        // (at d = 64 the last 32-column chunk also covers 16 allocated
+        // columns past the accumulator, which nothing reads)
 #pragma unroll 1
         for (int cc = 0; cc < (OW + 31) / 32; ++cc) {
           uint32_t o[32];

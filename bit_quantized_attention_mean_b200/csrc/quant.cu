@@ -292,11 +292,11 @@ quant_qk_kernel(const __half* __restrict__ q, const __half* __restrict__ k,
   // Per-block channel extremes, kept when this CTA's blocks fit in kFastBlocks:
   // fl32 rounding is monotonic, so over a block the largest |fl32(k - m_c)| of
   // channel c is taken at that channel's smallest or largest k.  Once the mean
-  // is known the block abs-max (and so the block scale) follows exactly,
-  // without a second pass over the rows.
-  // Used at d = 64, where it measured 8 % faster; at d = 128 the extra
-  // registers it needs cost the Q tiles (one kernel, one register budget)
-  // more than the shorter second pass gains.
+  // is known the block abs-max (and so the block scale) follows exactly, and
+  // the second pass needs no reduction over the rows it re-reads.
+  // Used at d = 64, where it measured 8 % faster; at d = 128 it measured
+  // 1-7 % slower (its extra registers spill in a kernel whose register budget
+  // the Q tiles share).
   constexpr bool kExtremes = D == 64;
   constexpr int kFastBlocks = kExtremes ? 4096 / D : 0;
   const int nb = kb1 - kb0;
