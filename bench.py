@@ -187,6 +187,20 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(busy)}
 
 
+def combined_roofline(d, pairs, attn_ms, p_int8, p_fp16, fp8):
+    """The attention kernel against its combined tensor roofline: 4 d ops per
+    unmasked (query, key) pair, half of them (QK^T) at the INT8 peak and half
+    (P V) at the FP16 peak, or at the 8-bit peak when P and V are FP8.
+    Peaks in TOPS / TFLOP/s, times in ms."""
+    p_pv = p_int8 if fp8 else p_fp16
+    t_roof_ms = (2.0 * d * pairs / (p_int8 * 1e12) + 2.0 * d * pairs / (p_pv * 1e12)) * 1e3
+    ops = 4.0 * d * pairs
+    return {"t_roof_ms": t_roof_ms,
+            "peak": ops / (t_roof_ms * 1e-3) / 1e12,          # equivalent combined peak
+            "achieved": ops / (attn_ms * 1e-3) / 1e12,
+            "frac": t_roof_ms / attn_ms}
+
+
 def secondary_ceilings(d, pairs, attn_ms, t_roof_ms, fp8, sms, sm_mhz):
     """The two further bars of the attention kernel: the fraction of the
     datasheet dense peaks (QK at INT8, P V at FP16 or FP8), and the exp2
@@ -520,12 +534,8 @@ def run_ours(args, w):
                    f"best of 10)" if p_int8_meas else
                    f"P_int8 = {INT8_OVER_FP16} x P_fp16 (nominal ratio)")
 
-        def roof_ms(pi8):
-            p_pv = pi8 if fp8 else p16   # FP8 P V runs at the 8-bit rate
-            return (2.0 * d * w.pairs() / (pi8 * 1e12) + 2.0 * d * w.pairs() / (p_pv * 1e12)) * 1e3
-        t_roof_ms = roof_ms(p8)
-        peak_eff = ops / (t_roof_ms * 1e-3) / 1e12
-        achieved = ops / (attn_avg_ms * 1e-3) / 1e12
+        roof = combined_roofline(d, w.pairs(), attn_avg_ms, p8, p16, fp8)
+        t_roof_ms, peak_eff, achieved = roof["t_roof_ms"], roof["peak"], roof["achieved"]
         traffic = None
         if NCU_TRAFFIC.get("attn_sha") == attn_source_hash() and \
                 NCU_TRAFFIC.get("workload") == w.name and \
@@ -554,7 +564,8 @@ def run_ours(args, w):
                 d, w.pairs(), attn_avg_ms, t_roof_ms, fp8,
                 torch.cuda.get_device_properties(dev).multi_processor_count,
                 clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0),
-                nominal_int8={"frac": roof_ms(p8_nominal) / attn_avg_ms,
+                nominal_int8={"frac": combined_roofline(d, w.pairs(), attn_avg_ms,
+                                                        p8_nominal, p16, fp8)["frac"],
                               "p_int8_tops": p8_nominal,
                               "note": "same kernel time, P_int8 = 2 x measured bf16 peak"}),
             "quant_hbm_gbs": quant_bytes / (quant_avg_ms * 1e-3) / 1e9,

@@ -96,7 +96,7 @@ def test_source_hash_ignores_comments_only():
 
 
 def test_secondary_ceilings_arithmetic():
-    """Closed forms: the LLM workload's 268,451,840 causal pairs at d = 128."""
+    """Closed forms: the LLM workload's 268,500,992 causal pairs at d = 128."""
     import bench
     pairs = 32 * 4096 * 4097 // 2
     c = bench.secondary_ceilings(128, pairs, attn_ms=0.1, t_roof_ms=0.05, fp8=False,
@@ -125,3 +125,40 @@ def test_cpu_baseline_sample_is_sized_by_pairs():
         per_row = w.pairs() / total
         if n < total:   # about the target, within one row
             assert abs(n * per_row - bench.CPU_BASELINE_PAIRS) <= per_row
+
+
+def test_workload_pair_counts_closed_forms():
+    """Unmasked (query, key) pairs: L^2 per head without a mask, L (L + 1) / 2
+    with the causal one; ops = 4 d pairs."""
+    from bit_quantized_attention_mean_b200 import inputs
+    W = inputs.WORKLOADS
+    assert W[1].pairs() == 2 * 256 * 256
+    assert W[2].pairs() == 32 * 4096 * 4097 // 2 == 268_500_992
+    assert W[3].pairs() == 2 * 24 * 16384 * 16384
+    assert W[4].pairs() == 4 * 32 * 8192 * 8193 // 2
+    assert W[5].pairs() == 16 * 32768 * 32769 // 2
+    assert 4 * W[5].d * W[5].pairs() == pytest.approx(4.398e12, rel=1e-3)
+    # bottom-right alignment when Lq != Lk: row i sees keys j <= i + Lk - Lq
+    assert inputs.visible_pairs(1, 1, 4, 6, True) == 3 + 4 + 5 + 6
+    assert inputs.visible_pairs(1, 1, 6, 4, True) == 0 + 0 + 1 + 2 + 3 + 4
+    assert inputs.visible_pairs(2, 3, 5, 7, False) == 2 * 3 * 5 * 7
+
+
+def test_combined_roofline_arithmetic():
+    """The LLM workload at the measured 1640.7 TFLOP/s bf16 peak and twice it
+    for INT8: t_roof = 2 d pairs / P_int8 + 2 d pairs / P_fp16 = 62.8 us, so
+    an attention kernel of 143.8 us is at 0.437 of it."""
+    import bench
+    pairs = 268_500_992
+    r = bench.combined_roofline(128, pairs, 0.1438, 3281.4, 1640.7, False)
+    assert r["t_roof_ms"] == pytest.approx(256 * pairs / 3281.4e12 * 1e3
+                                           + 256 * pairs / 1640.7e12 * 1e3)
+    assert r["t_roof_ms"] == pytest.approx(0.0628, abs=5e-5)
+    assert r["frac"] == pytest.approx(0.437, abs=1e-3)
+    # the reported fraction is achieved / equivalent peak, the same number
+    assert r["achieved"] / r["peak"] == pytest.approx(r["frac"])
+    # equal QK and P V work: the equivalent peak is the harmonic mean
+    assert r["peak"] == pytest.approx(2 / (1 / 3281.4 + 1 / 1640.7))
+    # FP8 P V runs at the 8-bit rate
+    r8 = bench.combined_roofline(128, pairs, 0.1438, 3281.4, 1640.7, True)
+    assert r8["t_roof_ms"] == pytest.approx(512 * pairs / 3281.4e12 * 1e3)
