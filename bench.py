@@ -187,6 +187,16 @@ class ClockSampler:
                 "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(busy)}
 
 
+def quant_algorithmic_bytes(B, H, Hkv, Lq, Lk, d, q_block_rows):
+    """Bytes the quantization step must move: each fp16 Q and K element read
+    once (2 B) and written once as int8 (1 B), plus the fp32 block scales of
+    Q and K and the fp32 K mean.  The second read of K (mean, then quantize)
+    is overhead, not part of it."""
+    elems = B * H * Lq * d + B * Hkv * Lk * d
+    scales = B * H * -(-Lq // q_block_rows) + B * Hkv * -(-Lk // 64)
+    return 3 * elems + 4 * scales + 4 * B * Hkv * d
+
+
 def combined_roofline(d, pairs, attn_ms, p_int8, p_fp16, fp8):
     """The attention kernel against its combined tensor roofline: 4 d ops per
     unmasked (query, key) pair, half of them (QK^T) at the INT8 peak and half
@@ -541,7 +551,7 @@ def run_ours(args, w):
                 NCU_TRAFFIC.get("workload") == w.name and \
                 NCU_TRAFFIC.get("q_block_rows", 128) == qbr and args.pv_accum == "f32":
             traffic = NCU_TRAFFIC.get("bytes_per_launch")
-        quant_bytes = 3 * (B * H * Lq + B * Hkv * Lk) * d + 4 * B * H * -(-Lq // qbr)
+        quant_bytes = quant_algorithmic_bytes(B, H, Hkv, Lq, Lk, d, qbr)
         result = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": n, "warmup": args.warmup, "ms_per_step": ms_per_step,

@@ -162,3 +162,18 @@ def test_combined_roofline_arithmetic():
     # FP8 P V runs at the 8-bit rate
     r8 = bench.combined_roofline(128, pairs, 0.1438, 3281.4, 1640.7, True)
     assert r8["t_roof_ms"] == pytest.approx(512 * pairs / 3281.4e12 * 1e3)
+
+
+def test_quant_algorithmic_bytes():
+    """The GQA workload: 4 (32 + 8) 8192 128 = 168 M elements at 3 B each, plus
+    the block scales (128-row Q, 64-row K blocks) and the K means, 4 B each."""
+    import bench
+    got = bench.quant_algorithmic_bytes(4, 32, 8, 8192, 8192, 128, 128)
+    elems = 4 * (32 + 8) * 8192 * 128
+    assert elems == 167_772_160
+    scales = 4 * 32 * 64 + 4 * 8 * 128
+    assert got == 3 * elems + 4 * scales + 4 * 4 * 8 * 128
+    assert got == pytest.approx(503.3e6, rel=1e-3)
+    # one Q scale per token at the long context
+    assert bench.quant_algorithmic_bytes(1, 16, 16, 32768, 32768, 128, 1) == \
+        3 * 2 * 16 * 32768 * 128 + 4 * (16 * 32768 + 16 * 512) + 4 * 16 * 128
